@@ -1,0 +1,97 @@
+"""Host-side checks of libhimuon (no GPU needed): the library loads, exports
+every entry point the header declares, rejects bad arguments without touching
+a device, and its tile planner numbers exactly the tiles of the oracle's
+tiling (split blocks first, tiles row-major from each block's top-left)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from tiled_newton_schulz_b200 import himuon
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_newton_schulz_b200 import build
+    build.build()
+    return himuon.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "himuon.h")).read()
+    return sorted(set(re.findall(r"HIMUON_API\s+[\w\s\*]+?\b(himuon_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 9
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(himuon.EXPORTS) <= set(names)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.himuon_version() == 1
+    assert himuon.status_string(0) == "ok"
+    assert "workspace" in himuon.status_string(-3)
+
+
+@pytest.mark.parametrize("shapes,splits,T", [
+    ([(10, 7)], None, 4),
+    ([(8, 24), (5, 5)], [(1, (8, 8, 8)), None], 4),
+    ([(300, 500), (128, 128)], None, 128),
+    ([(4096, 12288)], [(1, (4096, 4096, 4096))], 128),
+    ([(11008, 4096), (4096, 11008)], None, 512),
+    ([(10, 6)], [(0, (3, 7))], 4),
+    ([(9, 13)], None, 0),
+])
+def test_planner_matches_oracle_tiling(lib, shapes, splits, T):
+    got = himuon.plan_tiles(shapes, splits, T)
+    want = []
+    for i, shp in enumerate(shapes):
+        sp = splits[i] if splits else None
+        for (r0, c0, h, w) in oracle.split_blocks(shp, sp):
+            TT = max(h, w) if T <= 0 else T
+            for (tr, tc, th, tw) in oracle.tile_grid(h, w, TT):
+                want.append((i, r0 + tr, c0 + tc, th, tw))
+    assert got == want
+
+
+def test_llama7b_tile_count(lib):
+    from tiled_newton_schulz_b200 import inputs
+    wl = inputs.llama7b_set(1)
+    shapes = [(m.rows, m.cols) for m in wl.matrices]
+    splits = [m.split for m in wl.matrices]
+    assert len(himuon.plan_tiles(shapes, splits, 128)) == 395264 // 32
+    assert len(himuon.plan_tiles(shapes, splits, 256)) == 98816 // 32
+
+
+def test_invalid_arguments_are_rejected_on_the_host(lib):
+    p = himuon.params(128, (3.4445, -4.7750, 2.0315), steps=5)
+    m = (himuon.Mat * 1)(himuon.Mat(0, 16, 16, 16, himuon.BF16))   # null data
+    rc = lib.himuon_ns_tiled(m, m, 1, None, ctypes.byref(p), None, 0, None)
+    assert rc == -1
+    good = (himuon.Mat * 1)(himuon.Mat(0x1000, 16, 16, 8, himuon.BF16))   # ld < cols
+    assert lib.himuon_ns_tiled(good, good, 1, None, ctypes.byref(p), None, 0, None) == -1
+    bad_k = himuon.params(128, [(1.0, 0.0, 0.0)] * 17)
+    ok = (himuon.Mat * 1)(himuon.Mat(0x1000, 16, 16, 16, himuon.BF16))
+    assert lib.himuon_ns_tiled(ok, ok, 1, None, ctypes.byref(bad_k), None, 0, None) == -2
+    split = himuon._splits([(1, (8, 4))], 1)[0]    # sizes do not sum to 16
+    assert lib.himuon_workspace_size(ok, 1, split, ctypes.byref(p), 0) == -1
+
+
+def test_workspace_size_on_the_host(lib):
+    import torch
+    p = himuon.params(128, (3.4445, -4.7750, 2.0315), steps=5)
+    shapes = [(4096, 4096)]
+    mats = (himuon.Mat * 1)(himuon.Mat(0x1000, 4096, 4096, 4096, himuon.BF16))
+    assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p), 0) == 0       # on-chip path
+    p256 = himuon.params(256, (3.4445, -4.7750, 2.0315), steps=5)
+    need = lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p256), 0)
+    assert need > 256 * 256 * 8 * 256
+    pc = himuon.params(256, (3.4445, -4.7750, 2.0315), steps=5, chunk_bytes=64 << 20)
+    assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(pc), 0) <= 64 << 20

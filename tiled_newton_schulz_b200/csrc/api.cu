@@ -1,0 +1,867 @@
+// api.cu -- the C ABI of libhimuon: argument checks, the CMuon split, the tile
+// planner (cross-layer batching and memory-bounded chunking), a small plan
+// cache, and dispatch to the on-chip or the HBM-staged kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <list>
+#include <map>
+#include <memory>
+#include <string>
+#include <vector>
+
+#include "himuon.h"
+#include "layout.hpp"
+#include "resident.hpp"
+#include "staged.hpp"
+
+namespace himuon {
+
+// The device status word: kernels record the first device-side failure here
+// (bounded waits that gave up, inconsistent descriptors) instead of trapping.
+__device__ int g_device_status;
+
+namespace {
+
+int *status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  static int *cache[64] = {};
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int *>(p);
+  }
+  return cache[dev];
+}
+
+bool log_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("HIMUON_LOG");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+size_t elem_size(int32_t dt) { return dt == HIMUON_FP32 ? 4 : 2; }
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// ---------------------------------------------------------------- matrices and blocks
+struct CallMats {
+  int32_t n = 0;
+  const himuon_mat *role[kNumRoles] = {nullptr, nullptr, nullptr, nullptr};  // arrays of n, or null
+};
+
+struct HostBlock {
+  int32_t mat;
+  int64_t row0, col0, rows, cols;
+  int64_t T;            // tile edge
+  int64_t tiles_r, tiles_c, tile_begin;
+};
+
+int check_mat(const himuon_mat &m) {
+  if (!m.data || m.rows < 1 || m.cols < 1 || m.ld < m.cols) return HIMUON_ERR_INVALID;
+  if (m.rows > (int64_t)1 << 30 || m.cols > (int64_t)1 << 30) return HIMUON_ERR_UNSUPPORTED;
+  if (m.dtype < HIMUON_BF16 || m.dtype > HIMUON_FP32) return HIMUON_ERR_UNSUPPORTED;
+  return HIMUON_OK;
+}
+
+int check_params(const himuon_ns_params *p) {
+  if (!p || !p->coeffs) return HIMUON_ERR_INVALID;
+  if (p->steps < 1 || p->steps > kMaxSteps) return HIMUON_ERR_UNSUPPORTED;
+  if (p->compute < HIMUON_BF16 || p->compute > HIMUON_FP32) return HIMUON_ERR_UNSUPPORTED;
+  if (!(p->eps >= 0.f) || !(p->safety >= 0.f)) return HIMUON_ERR_INVALID;
+  for (int i = 0; i < 3 * p->steps; ++i)
+    if (!isfinite(p->coeffs[i])) return HIMUON_ERR_INVALID;
+  if (p->n_restart < 0 || (p->n_restart > 0 && !p->restart_at)) return HIMUON_ERR_INVALID;
+  if (p->chunk_bytes < 0) return HIMUON_ERR_INVALID;
+  return HIMUON_OK;
+}
+
+// CMuon split of every matrix into blocks, then the tile grid of each block.
+int make_blocks(const CallMats &cm, const himuon_split *splits, int64_t tile, std::vector<HostBlock> &out,
+                int64_t *n_tiles) {
+  out.clear();
+  const himuon_mat *base = nullptr;
+  for (int r = 0; r < kNumRoles && !base; ++r) base = cm.role[r];
+  int64_t next_tile = 0;
+  for (int32_t i = 0; i < cm.n; ++i) {
+    const himuon_mat &m = base[i];
+    std::vector<std::pair<int64_t, int64_t>> spans;  // (offset, size) along the split dim
+    int dim = 0;
+    if (splits && splits[i].nblocks > 1) {
+      const himuon_split &s = splits[i];
+      if ((s.dim != 0 && s.dim != 1) || !s.sizes) return HIMUON_ERR_INVALID;
+      dim = s.dim;
+      int64_t off = 0;
+      for (int b = 0; b < s.nblocks; ++b) {
+        if (s.sizes[b] < 1) return HIMUON_ERR_INVALID;
+        spans.push_back({off, s.sizes[b]});
+        off += s.sizes[b];
+      }
+      if (off != (dim == 0 ? m.rows : m.cols)) return HIMUON_ERR_INVALID;
+    } else {
+      spans.push_back({0, dim == 0 ? m.rows : m.cols});
+    }
+    for (auto &sp : spans) {
+      HostBlock b;
+      b.mat = i;
+      b.row0 = dim == 0 ? sp.first : 0;
+      b.col0 = dim == 1 ? sp.first : 0;
+      b.rows = dim == 0 ? sp.second : m.rows;
+      b.cols = dim == 1 ? sp.second : m.cols;
+      b.T = (tile <= 0) ? std::max(b.rows, b.cols) : tile;
+      b.tiles_r = (b.rows + b.T - 1) / b.T;
+      b.tiles_c = (b.cols + b.T - 1) / b.T;
+      b.tile_begin = next_tile;
+      next_tile += b.tiles_r * b.tiles_c;
+      out.push_back(b);
+    }
+  }
+  *n_tiles = next_tile;
+  return HIMUON_OK;
+}
+
+int check_call(const CallMats &cm, const himuon_split *splits) {
+  if (cm.n < 1) return HIMUON_ERR_INVALID;
+  const himuon_mat *base = nullptr;
+  for (int r = 0; r < kNumRoles && !base; ++r) base = cm.role[r];
+  if (!base) return HIMUON_ERR_INVALID;
+  for (int r = 0; r < kNumRoles; ++r) {
+    if (!cm.role[r]) continue;
+    for (int32_t i = 0; i < cm.n; ++i) {
+      const int rc = check_mat(cm.role[r][i]);
+      if (rc) return rc;
+      if (cm.role[r][i].rows != base[i].rows || cm.role[r][i].cols != base[i].cols) return HIMUON_ERR_INVALID;
+    }
+  }
+  (void)splits;
+  return HIMUON_OK;
+}
+
+// ---------------------------------------------------------------- plans
+enum PathKind { kPathResident = 0, kPathStaged = 1 };
+
+struct TileClass {
+  int64_t n, m;          // padded iterate shape (n <= m)
+  bool padded;           // some tile of the class is smaller than n x m
+  std::vector<DevTile> tiles;
+  int64_t dev_offset;    // index of the class's first DevTile in the device table
+};
+
+struct Plan {
+  int device = -1;
+  PathKind path = kPathStaged;
+  std::vector<HostBlock> blocks;
+  int64_t n_tiles = 0;
+  std::vector<TileClass> classes;
+  void *dev = nullptr;            // [DevBlock...][CUtensorMap...][DevTile...]
+  DevBlock *d_blocks = nullptr;
+  CUtensorMap *d_tmaps = nullptr;
+  DevTile *d_tiles = nullptr;
+  ~Plan() {
+    if (dev) cudaFree(dev);
+  }
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a bf16 block: box 64 columns x 128 rows, 128-byte swizzle,
+// zero fill outside the block (the zero padding of ragged tiles).
+bool make_block_map(CUtensorMap *map, void *ptr, int64_t rows, int64_t cols, int64_t ld) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+void *block_ptr(const himuon_mat &m, const HostBlock &b) {
+  return static_cast<char *>(m.data) + (b.row0 * m.ld + b.col0) * static_cast<int64_t>(elem_size(m.dtype));
+}
+
+bool resident_ok(const CallMats &cm, const std::vector<HostBlock> &blocks, const himuon_ns_params &p) {
+  if (p.compute == HIMUON_FP32) return false;
+  for (int r = 0; r < kNumRoles; ++r) {
+    if (!cm.role[r]) continue;
+    for (int32_t i = 0; i < cm.n; ++i) {
+      const himuon_mat &m = cm.role[r][i];
+      if (m.dtype != HIMUON_BF16) return false;
+      if ((m.ld * 2) % 16 != 0) return false;
+    }
+  }
+  for (const HostBlock &b : blocks) {
+    const bool single = b.T >= std::max(b.rows, b.cols) && std::max(b.rows, b.cols) <= 128;
+    if (!(b.T == 128 || single)) return false;
+    for (int r = 0; r < kNumRoles; ++r) {
+      if (!cm.role[r]) continue;
+      if (reinterpret_cast<uintptr_t>(block_ptr(cm.role[r][b.mat], b)) % 16 != 0) return false;
+    }
+  }
+  return true;
+}
+
+std::string plan_key(int device, int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params &p) {
+  std::string k;
+  auto put = [&k](const void *d, size_t n) { k.append(static_cast<const char *>(d), n); };
+  put(&device, sizeof device);
+  put(&op, sizeof op);
+  put(&cm.n, sizeof cm.n);
+  put(&p.tile, sizeof p.tile);
+  put(&p.compute, sizeof p.compute);
+  for (int r = 0; r < kNumRoles; ++r) {
+    const int present = cm.role[r] ? 1 : 0;
+    put(&present, sizeof present);
+    if (!present) continue;
+    for (int32_t i = 0; i < cm.n; ++i) {
+      const himuon_mat &m = cm.role[r][i];
+      put(&m.data, sizeof m.data);
+      put(&m.rows, sizeof m.rows);
+      put(&m.cols, sizeof m.cols);
+      put(&m.ld, sizeof m.ld);
+      put(&m.dtype, sizeof m.dtype);
+    }
+  }
+  for (int32_t i = 0; i < cm.n; ++i) {
+    const int32_t nb = (splits && splits[i].nblocks > 1) ? splits[i].nblocks : 0;
+    put(&nb, sizeof nb);
+    if (nb) {
+      put(&splits[i].dim, sizeof splits[i].dim);
+      put(splits[i].sizes, sizeof(int64_t) * nb);
+    }
+  }
+  return k;
+}
+
+struct PlanCache {
+  std::list<std::pair<std::string, std::shared_ptr<Plan>>> lru;
+  std::map<std::string, std::list<std::pair<std::string, std::shared_ptr<Plan>>>::iterator> index;
+  static constexpr size_t kCap = 32;
+};
+PlanCache &cache() {
+  static PlanCache *c = new PlanCache();  // never destroyed: avoids freeing at exit after the context is gone
+  return *c;
+}
+
+int build_plan(int device, int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params &p,
+               std::shared_ptr<Plan> &out) {
+  auto plan = std::make_shared<Plan>();
+  plan->device = device;
+  int rc = make_blocks(cm, splits, op == HIMUON_OP_NS_FULL || op == HIMUON_OP_GRAM_NS ? 0 : p.tile, plan->blocks,
+                       &plan->n_tiles);
+  if (rc) return rc;
+  const bool resident = op != HIMUON_OP_GRAM_NS && resident_ok(cm, plan->blocks, p);
+  plan->path = resident ? kPathResident : kPathStaged;
+
+  std::vector<DevBlock> dblocks(plan->blocks.size());
+  std::vector<CUtensorMap> tmaps;
+  for (size_t bi = 0; bi < plan->blocks.size(); ++bi) {
+    const HostBlock &b = plan->blocks[bi];
+    DevBlock &d = dblocks[bi];
+    memset(&d, 0, sizeof d);
+    d.tile_begin = b.tile_begin;
+    d.tiles_r = static_cast<int32_t>(b.tiles_r);
+    d.tiles_c = static_cast<int32_t>(b.tiles_c);
+    d.rows = static_cast<int32_t>(b.rows);
+    d.cols = static_cast<int32_t>(b.cols);
+    d.T = resident ? 128 : static_cast<int32_t>(b.T);
+    d.mat = b.mat;
+    for (int r = 0; r < kNumRoles; ++r) {
+      d.tmap[r] = -1;
+      if (!cm.role[r]) continue;
+      const himuon_mat &m = cm.role[r][b.mat];
+      d.ptr[r] = block_ptr(m, b);
+      d.ld[r] = m.ld;
+      d.dtype[r] = m.dtype;
+      if (resident) {
+        CUtensorMap tm;
+        if (!make_block_map(&tm, d.ptr[r], b.rows, b.cols, m.ld)) return HIMUON_ERR_CUDA;
+        d.tmap[r] = static_cast<int32_t>(tmaps.size());
+        tmaps.push_back(tm);
+      }
+    }
+  }
+  std::vector<DevTile> dtiles;
+  if (!resident) {
+    // shape classes of the staged path: padded (n, m), n <= m, multiples of 128
+    std::map<std::pair<int64_t, int64_t>, size_t> cls;
+    for (size_t bi = 0; bi < plan->blocks.size(); ++bi) {
+      const HostBlock &b = plan->blocks[bi];
+      for (int64_t tr = 0; tr < b.tiles_r; ++tr)
+        for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
+          DevTile t;
+          t.block = static_cast<int32_t>(bi);
+          t.r0 = static_cast<int32_t>(tr * b.T);
+          t.c0 = static_cast<int32_t>(tc * b.T);
+          t.h = static_cast<int32_t>(std::min(b.T, b.rows - t.r0));
+          t.w = static_cast<int32_t>(std::min(b.T, b.cols - t.c0));
+          t.transposed = t.h > t.w ? 1 : 0;
+          const int64_t n = round_up(std::min(t.h, t.w), 128), m = round_up(std::max(t.h, t.w), 128);
+          auto key = std::make_pair(n, m);
+          auto it = cls.find(key);
+          if (it == cls.end()) {
+            it = cls.emplace(key, plan->classes.size()).first;
+            TileClass c;
+            c.n = n;
+            c.m = m;
+            c.padded = false;
+            plan->classes.push_back(c);
+          }
+          TileClass &c = plan->classes[it->second];
+          if (std::min(t.h, t.w) != n || std::max(t.h, t.w) != m) c.padded = true;
+          c.tiles.push_back(t);
+        }
+    }
+    for (TileClass &c : plan->classes) {
+      c.dev_offset = static_cast<int64_t>(dtiles.size());
+      dtiles.insert(dtiles.end(), c.tiles.begin(), c.tiles.end());
+    }
+  }
+  // one device buffer: blocks | tensor maps (64-byte aligned) | tiles
+  const size_t sb = round_up(sizeof(DevBlock) * dblocks.size(), 128);
+  const size_t st = round_up(sizeof(CUtensorMap) * tmaps.size(), 128);
+  const size_t stl = sizeof(DevTile) * dtiles.size();
+  const size_t total = sb + st + stl + 128;
+  std::vector<char> host(total, 0);
+  memcpy(host.data(), dblocks.data(), sizeof(DevBlock) * dblocks.size());
+  if (!tmaps.empty()) memcpy(host.data() + sb, tmaps.data(), sizeof(CUtensorMap) * tmaps.size());
+  if (!dtiles.empty()) memcpy(host.data() + sb + st, dtiles.data(), stl);
+  if (cudaMalloc(&plan->dev, total) != cudaSuccess) return HIMUON_ERR_CUDA;
+  if (cudaMemcpy(plan->dev, host.data(), total, cudaMemcpyHostToDevice) != cudaSuccess) return HIMUON_ERR_CUDA;
+  plan->d_blocks = static_cast<DevBlock *>(plan->dev);
+  plan->d_tmaps = reinterpret_cast<CUtensorMap *>(static_cast<char *>(plan->dev) + sb);
+  plan->d_tiles = reinterpret_cast<DevTile *>(static_cast<char *>(plan->dev) + sb + st);
+  if (log_enabled()) {
+    fprintf(stderr, "[himuon] plan: op=%d path=%s blocks=%zu tiles=%lld classes=%zu tmaps=%zu\n", op,
+            resident ? "resident" : "staged", plan->blocks.size(), (long long)plan->n_tiles, plan->classes.size(),
+            tmaps.size());
+    for (const TileClass &c : plan->classes)
+      fprintf(stderr, "[himuon]   class n=%lld m=%lld tiles=%zu padded=%d\n", (long long)c.n, (long long)c.m,
+              c.tiles.size(), (int)c.padded);
+  }
+  out = plan;
+  return HIMUON_OK;
+}
+
+int get_plan(int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params &p,
+             std::shared_ptr<Plan> &out) {
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return HIMUON_ERR_NO_DEVICE;
+  const std::string key = plan_key(device, op, cm, splits, p);
+  PlanCache &c = cache();
+  auto it = c.index.find(key);
+  if (it != c.index.end()) {
+    c.lru.splice(c.lru.begin(), c.lru, it->second);
+    out = it->second->second;
+    return HIMUON_OK;
+  }
+  std::shared_ptr<Plan> plan;
+  const int rc = build_plan(device, op, cm, splits, p, plan);
+  if (rc) return rc;
+  c.lru.emplace_front(key, plan);
+  c.index[key] = c.lru.begin();
+  while (c.lru.size() > PlanCache::kCap) {
+    c.index.erase(c.lru.back().first);
+    c.lru.pop_back();
+  }
+  out = plan;
+  return HIMUON_OK;
+}
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return HIMUON_ERR_NO_DEVICE;
+  }
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return HIMUON_ERR_NO_DEVICE;
+  return major == 10 ? HIMUON_OK : HIMUON_ERR_NO_DEVICE;
+}
+
+// ---------------------------------------------------------------- workspace layout
+struct WsLayout {
+  size_t x32a, x32b, x16a, x16b, a32, a16, b32, b16, q32, q16a, q16b, z32, z16, rz32, rz16, partial, total;
+};
+
+WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, bool gram) {
+  WsLayout L;
+  memset(&L, 0, sizeof L);
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t o = off;
+    off += round_up(static_cast<int64_t>(bytes), 256);
+    return o;
+  };
+  const size_t nm = static_cast<size_t>(n * m * count), nn = static_cast<size_t>(n * n * count);
+  const bool f32 = compute == HIMUON_FP32;
+  L.x32a = take(4 * nm);
+  if (f32) L.x32b = take(4 * nm);
+  else {
+    L.x16a = take(2 * nm);
+    L.x16b = take(2 * nm);
+  }
+  L.a32 = take(4 * nn);
+  if (!f32) L.a16 = take(2 * nn);
+  if (!gram) {
+    if (f32) L.b32 = take(4 * nn);
+    else L.b16 = take(2 * nn);
+  } else {
+    L.q32 = take(4 * nn);
+    L.z32 = take(4 * nn);
+    L.rz32 = take(4 * nn);
+    if (f32) L.b32 = take(4 * nn);   // second Q buffer
+    else {
+      L.q16a = take(2 * nn);
+      L.q16b = take(2 * nn);
+      L.z16 = take(2 * nn);
+      L.rz16 = take(2 * nn);
+    }
+  }
+  const int64_t parts = (std::max(n, m) + 31) / 32;
+  L.partial = take(4 * parts * count);
+  L.total = off;
+  return L;
+}
+
+size_t chunk_limit(size_t ws_bytes, const himuon_ns_params &p) {
+  size_t lim = ws_bytes;
+  if (p.chunk_bytes > 0 && static_cast<size_t>(p.chunk_bytes) < lim) lim = static_cast<size_t>(p.chunk_bytes);
+  return lim;
+}
+
+// Tiles per chunk of a class under the limit (0 if even one tile does not fit).
+int64_t chunk_tiles(const TileClass &c, size_t limit, int compute, bool gram) {
+  const size_t one = ws_layout(c.n, c.m, 1, compute, gram).total;
+  int64_t k = static_cast<int64_t>(limit / one);
+  k = std::min<int64_t>(k, static_cast<int64_t>(c.tiles.size()));
+  k = std::min<int64_t>(k, 65535);
+  while (k > 0 && ws_layout(c.n, c.m, k, compute, gram).total > limit) --k;
+  return k;
+}
+
+int64_t staged_ws_bytes(const Plan &plan, int compute, bool gram) {
+  int64_t need = 0;
+  for (const TileClass &c : plan.classes)
+    need = std::max<int64_t>(need, static_cast<int64_t>(ws_layout(c.n, c.m, 1, compute, gram).total));
+  return need;
+}
+
+// ---------------------------------------------------------------- staged drivers
+#define HIMUON_TRY(x)                      \
+  do {                                     \
+    cudaError_t e_ = (x);                  \
+    if (e_ != cudaSuccess) return HIMUON_ERR_CUDA; \
+  } while (0)
+
+struct Ops {
+  int compute;
+  int32_t op16;   // operand dtype of the 16-bit copies
+  int *status;
+  cudaStream_t stream;
+  // acc = A op(B), batched; A, B given by (pointer, rows, cols) of 16-bit or fp32 storage
+  int mm(void *a, int64_t ar, int64_t ac, void *b, int64_t br, int64_t bc, int b_trans, int64_t M, int64_t N,
+         int64_t K, int64_t batch, const Epilogue &ep) const {
+    const int32_t dt = compute == HIMUON_FP32 ? HIMUON_FP32 : op16;
+    Batch A{a, ar, ac, ar * ac, dt}, B{b, br, bc, br * bc, dt};
+    cudaError_t e = compute == HIMUON_FP32 ? gemm_simt(A, B, b_trans, M, N, K, batch, ep, stream)
+                                           : gemm_tc(A, B, b_trans, M, N, K, batch, ep, status, stream);
+    return e == cudaSuccess ? HIMUON_OK : HIMUON_ERR_CUDA;
+  }
+};
+
+Epilogue epi(float alpha, float beta, const float *c32, float *out32, void *out16, int32_t dt) {
+  Epilogue e;
+  e.alpha = alpha;
+  e.beta = beta;
+  e.c32 = c32;
+  e.out32 = out32;
+  e.out16 = out16;
+  e.out16_dtype = dt;
+  e.diag = 0.f;
+  return e;
+}
+
+int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, float lr, void *ws, size_t ws_bytes,
+               cudaStream_t stream) {
+  const bool gram = op == HIMUON_OP_GRAM_NS;
+  const bool step = op == HIMUON_OP_MOMENTUM_STEP;
+  const int compute = p.compute;
+  const bool f32 = compute == HIMUON_FP32;
+  const size_t limit = chunk_limit(ws_bytes, p);
+  Ops ops{compute, compute == HIMUON_FP16 ? HIMUON_FP16 : HIMUON_BF16, status_ptr(), stream};
+  const int32_t dt16 = ops.op16;
+  const float safety = p.safety > 0.f ? p.safety : 1.f;
+  char *W = static_cast<char *>(ws);
+  for (const TileClass &c : plan.classes) {
+    const int64_t per = chunk_tiles(c, limit, compute, gram);
+    if (per < 1) return HIMUON_ERR_WORKSPACE;
+    const int64_t n = c.n, m = c.m;
+    for (int64_t t0 = 0; t0 < static_cast<int64_t>(c.tiles.size()); t0 += per) {
+      const int64_t bc = std::min<int64_t>(per, static_cast<int64_t>(c.tiles.size()) - t0);
+      const WsLayout L = ws_layout(n, m, bc, compute, gram);
+      float *x32[2] = {reinterpret_cast<float *>(W + L.x32a), f32 ? reinterpret_cast<float *>(W + L.x32b) : nullptr};
+      void *x16[2] = {f32 ? nullptr : W + L.x16a, f32 ? nullptr : W + L.x16b};
+      float *a32 = reinterpret_cast<float *>(W + L.a32);
+      void *a16 = f32 ? nullptr : W + L.a16;
+      const DevTile *tiles = plan.d_tiles + c.dev_offset + t0;
+      if (c.padded) HIMUON_TRY(cudaMemsetAsync(x32[0], 0, sizeof(float) * n * m * bc, stream));
+      PackArgs pk;
+      pk.blocks = plan.d_blocks;
+      pk.tiles = tiles;
+      pk.n_tiles = bc;
+      pk.n = n;
+      pk.m = m;
+      pk.x32 = x32[0];
+      pk.partial = reinterpret_cast<float *>(W + L.partial);
+      pk.rows_per_part = 32;
+      pk.parts = static_cast<int32_t>((std::max(n, m) + 31) / 32);
+      pk.mode = step ? 1 : 0;
+      pk.mu = mu;
+      HIMUON_TRY(launch_pack(pk, stream));
+      NormArgs na;
+      na.n_tiles = bc;
+      na.elems = n * m;
+      na.x32 = x32[0];
+      na.x16 = x16[0];
+      na.x16_dtype = dt16;
+      na.partial = pk.partial;
+      na.parts = pk.parts;
+      na.eps = p.eps;
+      na.safety = safety;
+      HIMUON_TRY(launch_normalize(na, stream));
+      int cur = 0;  // which x buffer holds the current operand
+      float *xfinal = x32[0];
+      int rc = HIMUON_OK;
+      // operand views: fp32 path reads the fp32 buffers directly
+      auto xop = [&](int i) -> void * { return f32 ? static_cast<void *>(x32[i]) : x16[i]; };
+      if (!gram) {
+        void *bop = f32 ? static_cast<void *>(W + L.b32) : W + L.b16;
+        for (int t = 0; t < p.steps && rc == HIMUON_OK; ++t) {
+          const float a = p.coeffs[3 * t], b = p.coeffs[3 * t + 1], cc = p.coeffs[3 * t + 2];
+          // A = X X^T
+          rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, epi(1.f, 0.f, nullptr, a32, a16, dt16));
+          if (rc) break;
+          // B' = b A + c A A + (a - 1) I
+          Epilogue e2 = epi(cc, b, a32, f32 ? static_cast<float *>(bop) : nullptr, f32 ? nullptr : bop, dt16);
+          e2.diag = a - 1.f;
+          rc = ops.mm(f32 ? static_cast<void *>(a32) : a16, n, n, f32 ? static_cast<void *>(a32) : a16, n, n, 0, n, n,
+                      n, bc, e2);
+          if (rc) break;
+          // X = a X + B X = X + B' X  (fp32 master in place; operand copy ping-pongs)
+          if (f32) {
+            rc = ops.mm(bop, n, n, x32[cur], n, m, 0, n, m, n, bc, epi(1.f, 1.f, x32[cur], x32[1 - cur], nullptr, dt16));
+            cur = 1 - cur;
+            xfinal = x32[cur];
+          } else {
+            rc = ops.mm(bop, n, n, x16[cur], n, m, 0, n, m, n, bc, epi(1.f, 1.f, x32[0], x32[0], x16[1 - cur], dt16));
+            cur = 1 - cur;
+          }
+        }
+      } else {
+        // Gram NS (Algorithm 3): R = X X^T, Q = I; restarts X <- Q X
+        float *r32 = a32, *q32 = reinterpret_cast<float *>(W + L.q32), *z32 = reinterpret_cast<float *>(W + L.z32);
+        float *rz32 = reinterpret_cast<float *>(W + L.rz32);
+        float *q32b = f32 ? reinterpret_cast<float *>(W + L.b32) : nullptr;
+        void *r16 = a16, *z16 = f32 ? nullptr : W + L.z16, *rz16 = f32 ? nullptr : W + L.rz16;
+        void *q16[2] = {f32 ? nullptr : W + L.q16a, f32 ? nullptr : W + L.q16b};
+        float *qf[2] = {q32, f32 ? q32b : q32};
+        int qc = 0;
+        auto rop = [&]() -> void * { return f32 ? static_cast<void *>(r32) : r16; };
+        auto zop = [&]() -> void * { return f32 ? static_cast<void *>(z32) : z16; };
+        auto rzop = [&]() -> void * { return f32 ? static_cast<void *>(rz32) : rz16; };
+        auto qop = [&](int i) -> void * { return f32 ? static_cast<void *>(qf[i]) : q16[i]; };
+        bool q_identity = true;
+        rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, epi(1.f, 0.f, nullptr, r32, r16, dt16));
+        for (int t = 1; t <= p.steps && rc == HIMUON_OK; ++t) {
+          const float a = p.coeffs[3 * (t - 1)], b = p.coeffs[3 * (t - 1) + 1], cc = p.coeffs[3 * (t - 1) + 2];
+          bool restart = false;
+          for (int i = 0; i < p.n_restart; ++i) restart |= p.restart_at[i] == t;
+          if (restart) {
+            if (!q_identity) {  // X <- Q X
+              if (f32) {
+                rc = ops.mm(qop(qc), n, n, x32[cur], n, m, 0, n, m, n, bc, epi(1.f, 0.f, nullptr, x32[1 - cur], nullptr, dt16));
+                cur = 1 - cur;
+                xfinal = x32[cur];
+              } else {
+                rc = ops.mm(qop(qc), n, n, x16[cur], n, m, 0, n, m, n, bc, epi(1.f, 0.f, nullptr, x32[0], x16[1 - cur], dt16));
+                cur = 1 - cur;
+              }
+              if (rc) break;
+              rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, epi(1.f, 0.f, nullptr, r32, r16, dt16));
+              if (rc) break;
+            }
+            q_identity = true;
+          }
+          // Z = b R + c R^2
+          rc = ops.mm(rop(), n, n, rop(), n, n, 0, n, n, n, bc, epi(cc, b, r32, z32, z16, dt16));
+          if (rc) break;
+          // Q <- Q Z + a Q
+          if (q_identity) {
+            HIMUON_TRY(launch_add_identity(z32, a, qf[qc], f32 ? nullptr : q16[qc], dt16, n, bc, stream));
+            q_identity = false;
+          } else {
+            rc = ops.mm(qop(qc), n, n, zop(), n, n, 0, n, n, n, bc,
+                        epi(1.f, a, qf[qc], qf[1 - qc], f32 ? nullptr : q16[1 - qc], dt16));
+            qc = 1 - qc;
+            if (rc) break;
+          }
+          if (t == p.steps) break;   // R_K is never used
+          // RZ <- R Z + a R
+          rc = ops.mm(rop(), n, n, zop(), n, n, 0, n, n, n, bc, epi(1.f, a, r32, rz32, rz16, dt16));
+          if (rc) break;
+          // R <- Z RZ + a RZ
+          rc = ops.mm(zop(), n, n, rzop(), n, n, 0, n, n, n, bc, epi(1.f, a, rz32, r32, r16, dt16));
+        }
+        if (rc == HIMUON_OK) {
+          // output Q X
+          if (f32) {
+            rc = ops.mm(qop(qc), n, n, x32[cur], n, m, 0, n, m, n, bc, epi(1.f, 0.f, nullptr, x32[1 - cur], nullptr, dt16));
+            xfinal = x32[1 - cur];
+          } else {
+            rc = ops.mm(qop(qc), n, n, x16[cur], n, m, 0, n, m, n, bc, epi(1.f, 0.f, nullptr, x32[0], nullptr, dt16));
+          }
+        }
+      }
+      if (rc) return rc;
+      UnpackArgs ua;
+      ua.blocks = plan.d_blocks;
+      ua.tiles = tiles;
+      ua.n_tiles = bc;
+      ua.n = n;
+      ua.m = m;
+      ua.x32 = xfinal;
+      ua.mode = step ? 1 : 0;
+      ua.lr = lr;
+      HIMUON_TRY(launch_unpack(ua, stream));
+    }
+  }
+  return HIMUON_OK;
+}
+
+int run_resident(const Plan &plan, int op, const himuon_ns_params &p, float mu, float lr, bool has_w, bool has_o,
+                 cudaStream_t stream) {
+  if (plan.n_tiles == 0) return HIMUON_OK;
+  ResidentArgs a;
+  memset(&a, 0, sizeof a);
+  a.blocks = plan.d_blocks;
+  a.tmaps = plan.d_tmaps;
+  a.n_blocks = static_cast<int32_t>(plan.blocks.size());
+  a.K = p.steps;
+  a.n_tiles = plan.n_tiles;
+  a.mode = op == HIMUON_OP_MOMENTUM_STEP ? 1 : 0;
+  a.has_w = has_w ? 1 : 0;
+  a.has_o = has_o ? 1 : 0;
+  a.op_fmt = p.compute == HIMUON_FP16 ? 0 : 1;
+  a.mu = mu;
+  a.lr = lr;
+  a.eps = p.eps;
+  a.safety = p.safety > 0.f ? p.safety : 1.f;
+  a.status = status_ptr();
+  make_resident_steps(a, p.coeffs, p.steps);
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, plan.device);
+  const int64_t want = (plan.n_tiles + 1) / 2;
+  const int grid = static_cast<int>(std::min<int64_t>(sms, want));
+  return launch_ns_resident(a, grid, stream) == cudaSuccess ? HIMUON_OK : HIMUON_ERR_CUDA;
+}
+
+int dispatch(int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params *p, float mu, float lr,
+             void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  rc = check_call(cm, splits);
+  if (rc) return rc;
+  rc = check_device();
+  if (rc) return rc;
+  std::shared_ptr<Plan> plan;
+  rc = get_plan(op, cm, splits, *p, plan);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (plan->path == kPathResident) {
+    const bool has_w = op == HIMUON_OP_MOMENTUM_STEP && cm.role[kRoleW];
+    const bool has_o = cm.role[kRoleOut] != nullptr;
+    return run_resident(*plan, op, *p, mu, lr, has_w, has_o, s);
+  }
+  const int64_t need = staged_ws_bytes(*plan, p->compute, op == HIMUON_OP_GRAM_NS);
+  if (!ws || static_cast<int64_t>(ws_bytes) < need) return HIMUON_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return HIMUON_ERR_ALIGNMENT;
+  return run_staged(*plan, op, *p, mu, lr, ws, ws_bytes, s);
+}
+
+}  // namespace
+}  // namespace himuon
+
+using namespace himuon;
+
+extern "C" {
+
+int himuon_ns_tiled(const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,
+                    const himuon_ns_params *p, void *ws, size_t ws_bytes, void *stream) {
+  if (!in || !out || !p) return HIMUON_ERR_INVALID;
+  CallMats cm;
+  cm.n = n;
+  cm.role[kRoleIn] = in;
+  cm.role[kRoleOut] = out;
+  const int op = (p->tile <= 0) ? HIMUON_OP_NS_FULL : HIMUON_OP_NS_TILED;
+  return dispatch(op, cm, splits, p, 0.f, 0.f, ws, ws_bytes, stream);
+}
+
+int himuon_ns_full(const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,
+                   const himuon_ns_params *p, void *ws, size_t ws_bytes, void *stream) {
+  if (!in || !out || !p) return HIMUON_ERR_INVALID;
+  CallMats cm;
+  cm.n = n;
+  cm.role[kRoleIn] = in;
+  cm.role[kRoleOut] = out;
+  return dispatch(HIMUON_OP_NS_FULL, cm, splits, p, 0.f, 0.f, ws, ws_bytes, stream);
+}
+
+int himuon_gram_ns(const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,
+                   const himuon_ns_params *p, void *ws, size_t ws_bytes, void *stream) {
+  if (!in || !out || !p) return HIMUON_ERR_INVALID;
+  CallMats cm;
+  cm.n = n;
+  cm.role[kRoleIn] = in;
+  cm.role[kRoleOut] = out;
+  return dispatch(HIMUON_OP_GRAM_NS, cm, splits, p, 0.f, 0.f, ws, ws_bytes, stream);
+}
+
+int himuon_momentum_step(const himuon_mat *W, const himuon_mat *M, const himuon_mat *G, int32_t n, float mu,
+                         float lr, const himuon_split *splits, const himuon_ns_params *p, const himuon_mat *update_out,
+                         void *ws, size_t ws_bytes, void *stream) {
+  if (!M || !G || !p || (!W && !update_out)) return HIMUON_ERR_INVALID;
+  if (!isfinite(mu) || !isfinite(lr)) return HIMUON_ERR_INVALID;
+  CallMats cm;
+  cm.n = n;
+  cm.role[kRoleIn] = M;
+  cm.role[kRoleG] = G;
+  cm.role[kRoleW] = W;
+  cm.role[kRoleOut] = update_out;
+  return dispatch(HIMUON_OP_MOMENTUM_STEP, cm, splits, p, mu, lr, ws, ws_bytes, stream);
+}
+
+int64_t himuon_workspace_size(const himuon_mat *mats, int32_t n, const himuon_split *splits,
+                              const himuon_ns_params *p, int32_t op) {
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (!mats || op < HIMUON_OP_NS_TILED || op > HIMUON_OP_MOMENTUM_STEP) return HIMUON_ERR_INVALID;
+  CallMats cm;
+  cm.n = n;
+  cm.role[kRoleIn] = mats;
+  cm.role[kRoleOut] = mats;
+  if (op == HIMUON_OP_MOMENTUM_STEP) cm.role[kRoleOut] = nullptr;
+  rc = check_call(cm, splits);
+  if (rc) return rc;
+  std::vector<HostBlock> blocks;
+  int64_t n_tiles = 0;
+  const int64_t tile = (op == HIMUON_OP_NS_FULL || op == HIMUON_OP_GRAM_NS) ? 0 : p->tile;
+  rc = make_blocks(cm, splits, tile, blocks, &n_tiles);
+  if (rc) return rc;
+  if (op != HIMUON_OP_GRAM_NS && resident_ok(cm, blocks, *p)) return 0;
+  // staged: one tile of the largest class is the minimum; a full chunk of every
+  // class makes the call run in one chunk per class.
+  int64_t need = 0;
+  std::map<std::pair<int64_t, int64_t>, int64_t> counts;
+  for (const HostBlock &b : blocks)
+    for (int64_t tr = 0; tr < b.tiles_r; ++tr)
+      for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
+        const int64_t h = std::min(b.T, b.rows - tr * b.T), w = std::min(b.T, b.cols - tc * b.T);
+        counts[{round_up(std::min(h, w), 128), round_up(std::max(h, w), 128)}] += 1;
+      }
+  for (auto &kv : counts) {
+    int64_t k = std::min<int64_t>(kv.second, 65535);
+    int64_t bytes = static_cast<int64_t>(ws_layout(kv.first.first, kv.first.second, k, p->compute,
+                                                   op == HIMUON_OP_GRAM_NS).total);
+    if (p->chunk_bytes > 0 && bytes > p->chunk_bytes)
+      bytes = std::max<int64_t>(p->chunk_bytes, static_cast<int64_t>(ws_layout(kv.first.first, kv.first.second, 1,
+                                                                                p->compute, op == HIMUON_OP_GRAM_NS)
+                                                                          .total));
+    need = std::max(need, bytes);
+  }
+  return need;
+}
+
+int himuon_get_device_status(void *stream) {
+  if (check_device() != HIMUON_OK) return HIMUON_ERR_NO_DEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HIMUON_ERR_CUDA;
+  int *p = status_ptr();
+  if (!p) return HIMUON_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return HIMUON_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return HIMUON_ERR_CUDA;
+  return v;
+}
+
+const char *himuon_status_string(int code) {
+  switch (code) {
+    case HIMUON_OK: return "ok";
+    case HIMUON_ERR_INVALID: return "invalid argument";
+    case HIMUON_ERR_UNSUPPORTED: return "unsupported dtype, tile size or step count";
+    case HIMUON_ERR_WORKSPACE: return "workspace too small";
+    case HIMUON_ERR_ALIGNMENT: return "pointer or row pitch not 16-byte aligned";
+    case HIMUON_ERR_CUDA: return "CUDA call failed";
+    case HIMUON_ERR_TIMEOUT: return "device wait timed out";
+    case HIMUON_ERR_DEVICE: return "inconsistent descriptor seen on the device";
+    case HIMUON_ERR_NO_DEVICE: return "no usable sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+int himuon_version(void) { return HIMUON_VERSION; }
+
+int64_t himuon_plan_tiles(const himuon_mat *mats, int32_t n, const himuon_split *splits, int32_t tile,
+                          int64_t *records, int64_t cap) {
+  if (!mats) return HIMUON_ERR_INVALID;
+  CallMats cm;
+  cm.n = n;
+  cm.role[kRoleIn] = mats;
+  int rc = check_call(cm, splits);
+  if (rc) return rc;
+  std::vector<HostBlock> blocks;
+  int64_t n_tiles = 0;
+  rc = make_blocks(cm, splits, tile, blocks, &n_tiles);
+  if (rc) return rc;
+  int64_t k = 0;
+  for (const HostBlock &b : blocks)
+    for (int64_t tr = 0; tr < b.tiles_r; ++tr)
+      for (int64_t tc = 0; tc < b.tiles_c; ++tc, ++k) {
+        if (!records || k >= cap) continue;
+        int64_t *r = records + 5 * k;
+        r[0] = b.mat;
+        r[1] = b.row0 + tr * b.T;
+        r[2] = b.col0 + tc * b.T;
+        r[3] = std::min(b.T, b.rows - tr * b.T);
+        r[4] = std::min(b.T, b.cols - tc * b.T);
+      }
+  return n_tiles;
+}
+
+}  // extern "C"

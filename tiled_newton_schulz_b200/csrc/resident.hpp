@@ -1,0 +1,43 @@
+// resident.hpp -- launch interface of the on-chip (T <= 128) tiled NS kernel.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "layout.hpp"
+
+namespace himuon {
+
+constexpr int kMaxSteps = 16;
+
+// Per-step scalars derived on the host from (a_t, b_t, c_t); see
+// make_resident_steps() for their meaning.
+struct ResidentStep {
+  float s;          // S = r(s * A) feeds MMA2
+  float beta;       // Bop = r(beta * D_P + am1 * I) feeds MMA3
+  float am1;        // a_t - 1
+  uint32_t neg2;    // MMA2 negates its A operand (c_t / beta < 0)
+  uint32_t acc2;    // MMA2 accumulates onto A (b_t != 0)
+};
+
+struct ResidentArgs {
+  const DevBlock *blocks;
+  const CUtensorMap *tmaps;
+  int32_t n_blocks;
+  int32_t K;
+  int64_t n_tiles;
+  int32_t mode;     // 0: NS in -> out; 1: momentum step
+  int32_t has_w, has_o;
+  int32_t op_fmt;   // tensor-core operand type: 0 fp16, 1 bf16
+  float mu, lr, eps, safety;
+  ResidentStep step[kMaxSteps];
+  int *status;
+};
+
+// Fills args.step[0..K) from K coefficient triples.
+void make_resident_steps(ResidentArgs &args, const float *coeffs, int K);
+
+int resident_smem_bytes();
+cudaError_t launch_ns_resident(const ResidentArgs &args, int grid, cudaStream_t stream);
+
+}  // namespace himuon

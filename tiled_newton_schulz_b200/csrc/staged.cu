@@ -1,0 +1,468 @@
+// staged.cu -- batched products and element passes of the HBM-staged path.
+//
+// Used for tiles larger than 128 x 128, for full-matrix NS and Gram NS, and
+// for fp32 arithmetic.  The iterate of every tile lives in workspace memory as
+// an fp32 master copy (x32) plus a 16-bit operand copy; each NS step
+// ("Gram Newton-Schulz" page, sec. 3, Algorithm 1) is three batched products
+// with fused epilogues:
+//     A  = X X^T                  -> A (fp32) and a 16-bit copy
+//     B  = b A + c (A A)          -> 16-bit B
+//     X  = a X + B X              -> X (fp32, in place) and a 16-bit copy
+// Tiles are zero-padded to multiples of 128 on both sides and transposed when
+// taller than wide; both leave the map unchanged (a zero border stays zero,
+// and NS(X^T) = NS(X)^T).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+#include "staged.hpp"
+
+namespace himuon {
+
+namespace {
+
+// ---------------------------------------------------------------- element access
+__device__ __forceinline__ float ld_elem(const void *p, int32_t dtype, int64_t i) {
+  if (dtype == HIMUON_BF16) return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+  if (dtype == HIMUON_FP16) return __half2float(static_cast<const __half *>(p)[i]);
+  return static_cast<const float *>(p)[i];
+}
+__device__ __forceinline__ void st_elem(void *p, int32_t dtype, int64_t i, float v) {
+  if (dtype == HIMUON_BF16) static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
+  else if (dtype == HIMUON_FP16) static_cast<__half *>(p)[i] = __float2half_rn(v);
+  else static_cast<float *>(p)[i] = v;
+}
+
+template <int NT>
+__device__ __forceinline__ float block_sum(float v, float *scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) scratch[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int i = 0; i < NT / 32; ++i) s += scratch[i];
+  }
+  return s;  // valid in thread 0
+}
+
+// ---------------------------------------------------------------- pack
+// grid (parts, tiles): CTA p copies source rows [p*rpp, (p+1)*rpp) of its tile.
+__global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
+  __shared__ float scratch[8];
+  const int64_t t = blockIdx.y;
+  const DevTile tl = a.tiles[t];
+  const DevBlock &b = a.blocks[tl.block];
+  const int32_t i0 = blockIdx.x * a.rows_per_part;
+  const int32_t i1 = min(tl.h, i0 + a.rows_per_part);
+  float *x = a.x32 + t * a.n * a.m;
+  float ss = 0.f;
+  if (i0 < i1) {
+    const int64_t cnt = static_cast<int64_t>(i1 - i0) * tl.w;
+    const void *src = b.ptr[kRoleIn];
+    const int64_t ld = b.ld[kRoleIn];
+    const int32_t dt = b.dtype[kRoleIn];
+    for (int64_t e = threadIdx.x; e < cnt; e += blockDim.x) {
+      const int32_t i = i0 + static_cast<int32_t>(e / tl.w), j = static_cast<int32_t>(e % tl.w);
+      const int64_t gi = static_cast<int64_t>(tl.r0 + i) * ld + tl.c0 + j;
+      float v = ld_elem(src, dt, gi);
+      if (a.mode == 1) {
+        const float g = ld_elem(b.ptr[kRoleG], b.dtype[kRoleG], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleG] + tl.c0 + j);
+        v = fmaf(a.mu, v, g);
+        st_elem(b.ptr[kRoleIn], dt, gi, v);
+      }
+      ss = fmaf(v, v, ss);
+      const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
+      x[xo] = v;
+    }
+  }
+  const float s = block_sum<256>(ss, scratch);
+  if (threadIdx.x == 0) a.partial[t * a.parts + blockIdx.x] = s;
+}
+
+// grid (chunks, tiles): rho from the partial sums (fixed order), then scale.
+__global__ void __launch_bounds__(256) normalize_kernel(const NormArgs a) {
+  const int64_t t = blockIdx.y;
+  float s = 0.f;
+  for (int p = 0; p < a.parts; ++p) s += a.partial[t * a.parts + p];
+  const float inv = 1.0f / ((sqrtf(s) + a.eps) * a.safety);
+  float *x = a.x32 + t * a.elems;
+  const int64_t per = (a.elems + gridDim.x - 1) / gridDim.x;
+  const int64_t e0 = blockIdx.x * per, e1 = min(a.elems, e0 + per);
+  for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+    const float v = x[e] * inv;
+    x[e] = v;
+    if (a.x16) st_elem(a.x16, a.x16_dtype, t * a.elems + e, v);
+  }
+}
+
+// grid (parts, tiles)
+__global__ void __launch_bounds__(256) unpack_kernel(const UnpackArgs a, int32_t rows_per_part) {
+  const int64_t t = blockIdx.y;
+  const DevTile tl = a.tiles[t];
+  const DevBlock &b = a.blocks[tl.block];
+  const int32_t i0 = blockIdx.x * rows_per_part, i1 = min(tl.h, i0 + rows_per_part);
+  if (i0 >= i1) return;
+  const float *x = a.x32 + t * a.n * a.m;
+  const int64_t cnt = static_cast<int64_t>(i1 - i0) * tl.w;
+  for (int64_t e = threadIdx.x; e < cnt; e += blockDim.x) {
+    const int32_t i = i0 + static_cast<int32_t>(e / tl.w), j = static_cast<int32_t>(e % tl.w);
+    const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
+    const float o = x[xo];
+    if (b.ptr[kRoleOut])
+      st_elem(b.ptr[kRoleOut], b.dtype[kRoleOut], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleOut] + tl.c0 + j, o);
+    if (a.mode == 1 && b.ptr[kRoleW]) {
+      const int64_t gi = static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleW] + tl.c0 + j;
+      const float w = ld_elem(b.ptr[kRoleW], b.dtype[kRoleW], gi);
+      st_elem(b.ptr[kRoleW], b.dtype[kRoleW], gi, fmaf(-a.lr, o, w));
+    }
+  }
+}
+
+__global__ void add_identity_kernel(const float *z, float a, float *q32, void *q16, int32_t dt, int64_t n,
+                                    int64_t total) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = (e / n) % n, c = e % n;
+    const float v = z[e] + (r == c ? a : 0.f);
+    q32[e] = v;
+    if (q16) st_elem(q16, dt, e, v);
+  }
+}
+
+__global__ void to16_kernel(const float *x, void *y, int32_t dt, int64_t total) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x)
+    st_elem(y, dt, e, x[e]);
+}
+
+// ---------------------------------------------------------------- epilogue
+struct EpiArgs {
+  float alpha, beta, diag;
+  const float *c32;
+  float *out32;
+  void *out16;
+  int32_t out16_dtype;
+  int64_t N;        // columns of the output matrices
+  int64_t stride;   // elements per output matrix (M * N)
+};
+
+// Write 8 consecutive outputs starting at element index `o` of the batch;
+// they sit in row `row`, columns col..col+7 of their matrix.
+__device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t row, int64_t col, const float *acc) {
+  float v[8];
+  if (e.c32) {
+    const float4 c0 = *reinterpret_cast<const float4 *>(e.c32 + o);
+    const float4 c1 = *reinterpret_cast<const float4 *>(e.c32 + o + 4);
+    const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = fmaf(e.alpha, acc[i], e.beta * cc[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = e.alpha * acc[i];
+  }
+  if (e.diag != 0.f && row >= col && row < col + 8) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] += (col + i == row) ? e.diag : 0.f;
+  }
+  if (e.out32) {
+    *reinterpret_cast<float4 *>(e.out32 + o) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(e.out32 + o + 4) = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  if (e.out16) {
+    uint4 u;
+    if (e.out16_dtype == HIMUON_FP16) {
+      __half2 *h = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+      *reinterpret_cast<uint4 *>(static_cast<__half *>(e.out16) + o) = u;
+    } else {
+      __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(e.out16) + o) = u;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- tcgen05 GEMM
+constexpr int kStages = 3;
+constexpr uint32_t kStageA = 16384, kStageB = 16384, kStageBytes = kStageA + kStageB;
+constexpr uint32_t kGemmSmem = kStages * kStageBytes + 128 + 1024;
+constexpr int kGemmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+
+struct GemmTcArgs {
+  int64_t K;
+  uint32_t idesc;
+  EpiArgs ep;
+  int *status;
+};
+
+template <int B_MN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                   const GemmTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + kStages * kStageBytes);
+  uint64_t *empty = full + kStages;
+  uint64_t *done = empty + kStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t n0 = blockIdx.x * 128, m0 = blockIdx.y * 128, z = blockIdx.z;
+  const int nk = static_cast<int>(a.K / 64);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      if (kb >= kStages && !mbar_wait(empty + s, ((kb / kStages) - 1) & 1, a.status)) break;
+      uint8_t *As = sm + s * kStageBytes, *Bs = As + kStageA;
+      mbar_arrive_expect_tx(full + s, kStageBytes);
+      tma_load_3d(As, &mapA, kb * 64, m0, z, full + s);
+      if (B_MN) {
+        tma_load_3d(Bs, &mapB, n0, kb * 64, z, full + s);
+        tma_load_3d(Bs + 8192, &mapB, n0 + 64, kb * 64, z, full + s);
+      } else {
+        tma_load_3d(Bs, &mapB, kb * 64, n0, z, full + s);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    bool ok = true;
+    for (int kb = 0; kb < nk && ok; ++kb) {
+      const int s = kb % kStages;
+      if (!(ok = mbar_wait(full + s, (kb / kStages) & 1, a.status))) break;
+      tc_fence_after();
+      const uint32_t as = smem_u32(sm + s * kStageBytes), bs = as + kStageA;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = sw128_desc(as + kk * 32, 16, 1024);
+        const uint64_t bd = B_MN ? sw128_desc(bs + kk * 2048, 8192, 1024) : sw128_desc(bs + kk * 32, 16, 1024);
+        mma_ss(tmem, ad, bd, a.idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(empty + s);
+    }
+    mma_commit(done);
+  } else if (warp >= 2) {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    if (mbar_wait(done, 0, a.status)) {
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const int64_t obase = z * a.ep.stride + static_cast<int64_t>(m0 + row) * a.ep.N + n0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float v[32];
+        tmem_ld32(taddr + 32 * i, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) epi_store8(a.ep, obase + 32 * i + 8 * j, m0 + row, n0 + 32 * i + 8 * j, v + 8 * j);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ---------------------------------------------------------------- fp32 SIMT GEMM
+constexpr int kSB = 64, kSK = 16;
+template <int BT>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(const float *A, const float *B, int64_t K, int64_t lda,
+                                                        int64_t ldb, int64_t sA, int64_t sB, EpiArgs ep) {
+  __shared__ float As[kSK][kSB + 4];
+  __shared__ float Bs[kSK][kSB + 4];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int64_t n0 = blockIdx.x * kSB, m0 = blockIdx.y * kSB, z = blockIdx.z;
+  A += z * sA;
+  B += z * sB;
+  float acc[4][4] = {};
+  for (int64_t k0 = 0; k0 < K; k0 += kSK) {
+    for (int e = threadIdx.x; e < kSB * kSK; e += 256) {
+      const int r = e / kSK, c = e % kSK;   // A: 64 rows x 16 k
+      As[c][r] = A[(m0 + r) * lda + k0 + c];
+      if (BT) Bs[c][r] = B[(n0 + r) * ldb + k0 + c];
+    }
+    if (!BT) {
+      for (int e = threadIdx.x; e < kSB * kSK; e += 256) {
+        const int r = e / kSB, c = e % kSB;  // B: 16 k rows x 64 cols
+        Bs[r][c] = B[(k0 + r) * ldb + n0 + c];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kSK; ++k) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[k][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = Bs[k][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t o = z * ep.stride + (m0 + ty * 4 + i) * ep.N + n0 + tx * 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float v = ep.alpha * acc[i][j];
+      if (ep.c32) v = fmaf(ep.beta, ep.c32[o + j], v);
+      if (m0 + ty * 4 + i == n0 + tx * 4 + j) v += ep.diag;
+      if (ep.out32) ep.out32[o + j] = v;
+      if (ep.out16) st_elem(ep.out16, ep.out16_dtype, o + j, v);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host helpers
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D map over a batch of row-major [batch][rows][cols] 16-bit matrices.
+bool make_batch_map(CUtensorMap *m, const Batch &b, int64_t batch, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const CUtensorMapDataType dt =
+      b.dtype == HIMUON_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(b.cols), static_cast<cuuint64_t>(b.rows),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(b.cols * 2), static_cast<cuuint64_t>(b.stride * 2)};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, dt, 3, b.ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+EpiArgs to_epi(const Epilogue &e, int64_t M, int64_t N) {
+  EpiArgs a;
+  a.alpha = e.alpha;
+  a.beta = e.beta;
+  a.diag = e.diag;
+  a.c32 = e.c32;
+  a.out32 = e.out32;
+  a.out16 = e.out16;
+  a.out16_dtype = e.out16_dtype;
+  a.N = N;
+  a.stride = M * N;
+  return a;
+}
+
+}  // namespace
+
+cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int64_t N, int64_t K, int64_t batch,
+                    const Epilogue &ep, int *status, cudaStream_t stream) {
+  if (M % 128 || N % 128 || K % 64 || batch < 1 || batch > 65535) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb;
+  if (!make_batch_map(&ma, A, batch, 64, 128)) return cudaErrorInvalidValue;
+  if (b_trans) {
+    if (!make_batch_map(&mb, B, batch, 64, 128)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_batch_map(&mb, B, batch, 64, 64)) return cudaErrorInvalidValue;
+  }
+  GemmTcArgs a;
+  a.K = K;
+  a.idesc = idesc_f16(128, 128, A.dtype == HIMUON_FP16 ? 0u : 1u, 0, b_trans ? 0u : 1u, 0);
+  a.ep = to_epi(ep, M, N);
+  a.status = status;
+  dim3 grid(static_cast<unsigned>(N / 128), static_cast<unsigned>(M / 128), static_cast<unsigned>(batch));
+  cudaError_t e;
+  if (b_trans) {
+    e = cudaFuncSetAttribute(gemm_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+    if (e != cudaSuccess) return e;
+    gemm_tc_kernel<0><<<grid, kGemmThreads, kGemmSmem, stream>>>(ma, mb, a);
+  } else {
+    e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+    if (e != cudaSuccess) return e;
+    gemm_tc_kernel<1><<<grid, kGemmThreads, kGemmSmem, stream>>>(ma, mb, a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_simt(const Batch &A, const Batch &B, int b_trans, int64_t M, int64_t N, int64_t K, int64_t batch,
+                      const Epilogue &ep, cudaStream_t stream) {
+  if (M % kSB || N % kSB || K % kSK || batch < 1 || batch > 65535) return cudaErrorInvalidValue;
+  dim3 grid(static_cast<unsigned>(N / kSB), static_cast<unsigned>(M / kSB), static_cast<unsigned>(batch));
+  const float *pa = static_cast<const float *>(A.ptr), *pb = static_cast<const float *>(B.ptr);
+  if (b_trans)
+    gemm_simt_kernel<1><<<grid, 256, 0, stream>>>(pa, pb, K, A.cols, B.cols, A.stride, B.stride, to_epi(ep, M, N));
+  else
+    gemm_simt_kernel<0><<<grid, 256, 0, stream>>>(pa, pb, K, A.cols, B.cols, A.stride, B.stride, to_epi(ep, M, N));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack(const PackArgs &a, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>(a.parts), static_cast<unsigned>(a.n_tiles));
+  pack_kernel<<<grid, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_normalize(const NormArgs &a, cudaStream_t stream) {
+  const int64_t chunks = (a.elems + 8191) / 8192;
+  dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(a.n_tiles));
+  normalize_kernel<<<grid, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack(const UnpackArgs &a, cudaStream_t stream) {
+  const int32_t rpp = 32;
+  const int64_t side = a.n > a.m ? a.n : a.m;   // a tile has at most max(n, m) rows
+  const int64_t parts = (side + rpp - 1) / rpp;
+  dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(a.n_tiles));
+  unpack_kernel<<<grid, 256, 0, stream>>>(a, rpp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_add_identity(const float *z32, float a, float *q32, void *q16, int32_t q16_dtype, int64_t n,
+                                int64_t batch, cudaStream_t stream) {
+  const int64_t total = n * n * batch;
+  const int blocks = static_cast<int>((total + 255) / 256 < 65535 ? (total + 255) / 256 : 65535);
+  add_identity_kernel<<<blocks, 256, 0, stream>>>(z32, a, q32, q16, q16_dtype, n, total);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_to16(const float *x32, void *x16, int32_t dtype, int64_t count, cudaStream_t stream) {
+  const int blocks = static_cast<int>((count + 255) / 256 < 65535 ? (count + 255) / 256 : 65535);
+  to16_kernel<<<blocks, 256, 0, stream>>>(x32, x16, dtype, count);
+  return cudaGetLastError();
+}
+
+}  // namespace himuon

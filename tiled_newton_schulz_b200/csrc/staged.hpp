@@ -1,0 +1,85 @@
+// staged.hpp -- HBM-staged batched path for tiles larger than 128 and for
+// full-matrix NS / Gram NS, plus the fp32 CUDA-core path.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "layout.hpp"
+
+namespace himuon {
+
+// A batch of equally shaped row-major matrices in workspace memory.
+struct Batch {
+  void *ptr;          // element (0,0) of matrix 0
+  int64_t rows, cols; // each matrix
+  int64_t stride;     // elements between consecutive matrices (= rows * cols)
+  int32_t dtype;      // himuon_dtype
+};
+
+// Epilogue of the batched products below:
+//   out32 = alpha * acc + beta * c32 + diag * I   (c32 may be null: beta ignored)
+//   out16 = 16-bit copy of out32 (operand dtype), optional
+struct Epilogue {
+  float alpha, beta;
+  float diag;       // added on the diagonal of each (square) output matrix
+  const float *c32;
+  float *out32;
+  void *out16;
+  int32_t out16_dtype;
+};
+
+// acc = A * B^T (b_trans = 1, B is N x K) or A * B (b_trans = 0, B is K x N),
+// for every matrix of the batch.  A: M x K.  Operands are 16-bit for the
+// tensor-core version and fp32 for the CUDA-core version.  M, N multiples of
+// 128 and K a multiple of 64 (the planner pads with zeros).
+cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int64_t N, int64_t K, int64_t batch,
+                    const Epilogue &ep, int *status, cudaStream_t stream);
+cudaError_t gemm_simt(const Batch &A, const Batch &B, int b_trans, int64_t M, int64_t N, int64_t K, int64_t batch,
+                      const Epilogue &ep, cudaStream_t stream);
+
+// ----------------------------------------------------------------- element passes
+struct PackArgs {
+  const DevBlock *blocks;
+  const DevTile *tiles;   // tiles of this chunk
+  int64_t n_tiles;
+  int64_t n, m;           // padded iterate shape (n <= m), row-major n x m per tile
+  float *x32;             // n_tiles * n * m
+  float *partial;         // n_tiles * parts
+  int32_t parts;          // partial sums per tile (row slices of the source tile)
+  int32_t rows_per_part;
+  int32_t mode;           // 0: NS input; 1: momentum (M' = mu M + G written back to M)
+  float mu;
+};
+cudaError_t launch_pack(const PackArgs &a, cudaStream_t stream);
+
+struct NormArgs {
+  int64_t n_tiles;
+  int64_t elems;          // n * m per tile
+  float *x32;
+  void *x16;              // optional 16-bit operand copy
+  int32_t x16_dtype;
+  const float *partial;
+  int32_t parts;
+  float eps, safety;
+};
+cudaError_t launch_normalize(const NormArgs &a, cudaStream_t stream);
+
+struct UnpackArgs {
+  const DevBlock *blocks;
+  const DevTile *tiles;
+  int64_t n_tiles;
+  int64_t n, m;
+  const float *x32;
+  int32_t mode;           // 0: write role Out; 1: momentum: W -= lr O (if W), O to role Out (if present)
+  float lr;
+};
+cudaError_t launch_unpack(const UnpackArgs &a, cudaStream_t stream);
+
+// q32/q16 <- z32 + a I  (n x n per matrix); used when Q = I in Gram NS
+cudaError_t launch_add_identity(const float *z32, float a, float *q32, void *q16, int32_t q16_dtype, int64_t n,
+                                int64_t batch, cudaStream_t stream);
+// 16-bit copy of an fp32 batch
+cudaError_t launch_to16(const float *x32, void *x16, int32_t dtype, int64_t count, cudaStream_t stream);
+
+}  // namespace himuon
