@@ -1,0 +1,406 @@
+"""Throughput of the tiled-NS optimizer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--tile 128] [--impl ours|reference]
+
+Workload (default): one full Muon step over every 2-D weight of a Llama-style
+7B shape (32 layers; fused QKV 4096x12288 split into three 4096x4096 blocks;
+O 4096x4096; gate/up 4096x11008; down 11008x4096): M <- 0.95 M + G,
+O = tiledNS_T(M) with K = 5 quintic steps, W <- W - 0.02 O, all bf16 in HBM
+(38.9 GB of W, M, G).  Synthetic inputs: M and G low-rank-plus-noise
+(U diag(1/i) V^T, rank 64, Haar U, V, + 0.01 N(0,1)), W = 0.02 N(0,1).
+
+A step is one himuon_momentum_step call over all matrices.  The inputs
+(38.9 GB) are far larger than L2 (126 MB), so no flush is needed between
+steps.  Time is taken with CUDA events on the launching stream; with N > 1
+every rank runs its own replica of the workload (the tiles are independent:
+no data-path collective) and the max over ranks is reported.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+QUINTIC = (3.4445, -4.7750, 2.0315)
+K_STEPS = 5
+MU, LR = 0.95, 0.02
+METRIC = "tiled-NS step: matrix elements/s"
+
+
+# ---------------------------------------------------------------- helpers
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def flops_per_tile(h: int, w: int, K: int) -> float:
+    """The pages' per-step count 2(2 alpha + 1) n^3 for an n x m tile, n <= m."""
+    n, m = min(h, w), max(h, w)
+    return K * (4.0 * m * n * n + 2.0 * n ** 3)
+
+
+def workload_tiles(shapes_splits, T):
+    tiles, flops = 0, 0.0
+    for (H, W), split in shapes_splits:
+        blocks = [(H, W)] if split is None else [((H, s) if split[0] == 1 else (s, W)) for s in split[1]]
+        for (h, w) in blocks:
+            for r0 in range(0, h, T):
+                for c0 in range(0, w, T):
+                    th, tw = min(T, h - r0), min(T, w - c0)
+                    tiles += 1
+                    flops += flops_per_tile(th, tw, K_STEPS)
+    return tiles, flops
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        loaded = [s for s in sm if mx and s > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload
+
+def llama7b_matrices(layers: int = 32):
+    from tiled_newton_schulz_b200.inputs import llama7b_set
+    wl = llama7b_set(layers)
+    return [((m.rows, m.cols), m.split) for m in wl.matrices]
+
+
+def make_state(device, seed_base: int, layers: int = 32):
+    import torch
+    from tiled_newton_schulz_b200.inputs import gaussian_torch, low_rank_plus_noise_torch
+    mats = llama7b_matrices(layers)
+    W, M, G = [], [], []
+    for i, ((H, Wd), _) in enumerate(mats):
+        W.append((gaussian_torch(H, Wd, seed_base + 3 * i, device, torch.float32) * 0.02).to(torch.bfloat16))
+        M.append(low_rank_plus_noise_torch(H, Wd, 64, 0.01, seed_base + 3 * i + 1, device))
+        G.append(low_rank_plus_noise_torch(H, Wd, 64, 0.01, seed_base + 3 * i + 2, device))
+    torch.cuda.synchronize(device)
+    return mats, W, M, G
+
+
+def cpu_oracle_sample(mats_state, T: int, budget_s: float):
+    """Oracle on tiles of layer 0 (strips of whole tiles) until the budget is used.
+
+    Returns (elements/s, elements, seconds, threads, description)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    W, M, G = mats_state
+    H, Wd = W.shape
+    cols = 16 * T            # one strip of 16 tiles per call (OpenMP over its tiles)
+    elems, t0, strips = 0, time.perf_counter(), 0
+    while True:
+        c0 = (strips % 2) * (Wd - cols)
+        sl = np.s_[0:T, c0:c0 + cols]
+        oracle.momentum_step(W[sl], M[sl], G[sl], MU, LR, T, [QUINTIC] * K_STEPS)
+        elems += T * cols
+        strips += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            break
+    desc = (f"{strips} strips of 16 {T}x{T} tiles from layer 0's O projection (fused momentum, "
+            f"K={K_STEPS} NS steps, weight update), fp64")
+    return elems / dt, elems, dt, oracle.num_threads(), desc
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    rng = np.random.default_rng(5)
+    T = args.tile
+    H, Wd = 4096, 4096
+    from tiled_newton_schulz_b200 import inputs
+    W = 0.02 * rng.standard_normal((T, 16 * T))
+    Mx = inputs.low_rank_plus_noise(T, 16 * T, inputs.sigma_inverse(64), 0.01, seed=1)
+    Gx = inputs.low_rank_plus_noise(T, 16 * T, inputs.sigma_inverse(64), 0.01, seed=2)
+    import oracle
+    oracle.build()
+    per_step = []
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.momentum_step(W, Mx, Gx, MU, LR, T, [QUINTIC] * K_STEPS)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            per_step.append(dt)
+    elems = T * 16 * T
+    total = sum(per_step)
+    value = elems * len(per_step) / total
+    mats = llama7b_matrices()
+    desc = (f"one strip of 16 {T}x{T} tiles per step (fused momentum, K={K_STEPS} NS steps, weight update) "
+            f"of the Llama-7B step workload, fp64, low-rank-plus-noise inputs")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(per_step),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"llama7b_32l_full_step_T{T}", "tile": T, "steps_K": K_STEPS,
+                   "matrices": len(mats), "sample_per_step_elements": elems},
+        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from tiled_newton_schulz_b200 import himuon as hm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    hm.load()
+
+    T = args.tile
+    compute = {"bf16": hm.BF16, "fp16": hm.FP16}[args.compute]
+    mats, W, M, G = make_state(device, seed_base=1000 * rank, layers=args.layers)
+    splits = [s for (_, s) in mats]
+    elements = sum(H * Wd for (H, Wd), _ in mats)
+    n_tiles, flops = workload_tiles(mats, T)
+    p = hm.params(T, QUINTIC, steps=K_STEPS, compute=compute)
+    ws_need = hm.workspace_size(M, p, hm.OP_MOMENTUM_STEP, splits)
+    ws = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=device) if ws_need else None
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        hm.momentum_step(W, M, G, MU, LR, p, splits=splits, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    st = hm.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {hm.status_string(st)}")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = hm.launch_count()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    launches = hm.launch_count() - launches0
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    st = hm.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {hm.status_string(st)}")
+    ms_step = ms / args.steps
+    value = world * elements / (ms_step / 1e3)
+    tflops = world * flops / (ms_step / 1e3) / 1e12
+
+    # end to end through the public API with host buffers (pinned), this rank's replica
+    e2e_value, h2d, d2h = None, 0, 0
+    if not args.no_e2e:
+        hW = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in W]
+        hM = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in M]
+        hG = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in G]
+        for h, d in zip(hW + hM + hG, W + M + G):
+            h.copy_(d)
+        h2d = sum(x.numel() * x.element_size() for x in hW + hM + hG)
+        d2h = sum(x.numel() * x.element_size() for x in hW + hM)
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            for d, h in zip(W + M + G, hW + hM + hG):
+                d.copy_(h, non_blocking=True)
+            step()
+            for h, d in zip(hW + hM, W + M):
+                h.copy_(d, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize(device)
+        ems = a0.elapsed_time(a1)
+        if world > 1:
+            t = torch.tensor([ems], device=device, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e_value = world * elements / (ems / e2e_steps / 1e3)
+        del hW, hM, hG
+
+    # CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        idx = 1  # layer 0, O projection (4096 x 4096)
+        sample = tuple(x[idx][:T].detach().double().cpu().numpy() for x in (W, M, G))
+        v, e, dt, threads, desc = cpu_oracle_sample(sample, T, args.cpu_budget)
+        cpu = {"value": v, "unit": "elements/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": round(dt, 2)}
+
+    peaks, peak_src = read_peaks()
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    peak_burst = float(peaks.get("bf16_tflops"))
+    # the step is a single launch of the on-chip kernel: launch duration = step time
+    achieved = flops / (ms_step / 1e3) / 1e12
+    prof = load_profile_traffic(T)
+    roofline = {
+        "bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
+        "traffic": prof, "kernel": "ns_resident_kernel",
+        "peak_source": f"bf16_tflops_sustained ({peak_src})",
+        "frac_of_burst_peak": achieved / peak_burst,
+        "flops_per_launch": flops, "flop_count": "nominal: 2(2a+1)n^3 per NS step per tile (a = m/n)",
+        "hbm_bytes_per_launch": 10 * elements,
+        "hbm_time_ms": 10 * elements / (float(peaks.get("hbm_gbs")) * 1e9) * 1e3,
+        "tensor_time_ms_sustained_peak": flops / (peak_sus * 1e12) * 1e3,
+    }
+    line = {
+        "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": args.compute, "data": "synthetic",
+        "config": {"workload": f"llama7b_{args.layers}l_full_step_T{T}", "tile": T, "steps_K": K_STEPS, "mu": MU, "lr": LR,
+                   "matrices": len(mats), "split_blocks": sum(len(s[1]) if s else 1 for s in splits),
+                   "tiles": n_tiles, "elements_per_gpu": elements, "storage": "bf16 W, M, G",
+                   "accumulate": "fp32",
+                   "l2": f"inputs {6 * elements / 1e9:.1f} GB per GPU >> 126 MB L2, no flush",
+                   "parallelism": f"replicas x{world} (independent tiles, no collective)"},
+        "tflops": tflops,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "elements/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def load_profile_traffic(T: int):
+    """DRAM bytes per launch of the on-chip kernel from the committed ncu
+    summary, or None when there is none or the kernel source changed since."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", f"ns_resident_llama7b_T{T}_traffic.json")
+    src = os.path.join(ROOT, "tiled_newton_schulz_b200", "csrc", "ns_resident.cu")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return d.get("dram_bytes_per_full_launch") if d.get("kernel_source_sha256_prefix") == sha else None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--tile", type=int, default=128)
+    ap.add_argument("--layers", type=int, default=32, help="transformer layers of the 7B shape set")
+    ap.add_argument("--compute", choices=["bf16", "fp16"], default="bf16")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -179,6 +179,13 @@ HIMUON_API const char *himuon_status_string(int code);
 HIMUON_API int himuon_version(void);
 
 /*
+ * Number of CUDA kernels this library has enqueued since it was loaded, on all
+ * devices and streams (a host-side counter, incremented at each launch; no
+ * device synchronisation).  For accounting in benchmarks and tests.
+ */
+HIMUON_API int64_t himuon_launch_count(void);
+
+/*
  * Host-side tile list of a call, for checking the planner against a reference
  * tiling.  Fills up to `cap` records of 5 int64 each:
  *     (matrix index, row0, col0, h, w)

@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <list>
 #include <map>
 #include <memory>
@@ -25,6 +26,9 @@ namespace himuon {
 // The device status word: kernels record the first device-side failure here
 // (bounded waits that gave up, inconsistent descriptors) instead of trapping.
 __device__ int g_device_status;
+
+static std::atomic<long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 namespace {
 
@@ -836,6 +840,8 @@ const char *himuon_status_string(int code) {
 }
 
 int himuon_version(void) { return HIMUON_VERSION; }
+
+int64_t himuon_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int64_t himuon_plan_tiles(const himuon_mat *mats, int32_t n, const himuon_split *splits, int32_t tile,
                           int64_t *records, int64_t cap) {

@@ -4,6 +4,9 @@
 
 namespace himuon {
 
+// Host-side count of kernels enqueued by the library (defined in api.cu).
+void count_launch();
+
 // Roles a matrix plays in a call.
 enum Role : int { kRoleIn = 0,   // NS input; momentum M (read, then M' written back)
                   kRoleOut = 1,  // NS output; update O of a momentum step

@@ -453,6 +453,7 @@ static cudaError_t launch_fmt(const ResidentArgs &args, int grid, cudaStream_t s
   cudaError_t e = cudaFuncSetAttribute(ns_resident_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
+  count_launch();
   ns_resident_kernel<F><<<grid, kThreads, kSmemBytes, stream>>>(args);
   return cudaGetLastError();
 }

@@ -408,10 +408,12 @@ cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int6
   if (b_trans) {
     e = cudaFuncSetAttribute(gemm_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
     if (e != cudaSuccess) return e;
+    count_launch();
     gemm_tc_kernel<0><<<grid, kGemmThreads, kGemmSmem, stream>>>(ma, mb, a);
   } else {
     e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
     if (e != cudaSuccess) return e;
+    count_launch();
     gemm_tc_kernel<1><<<grid, kGemmThreads, kGemmSmem, stream>>>(ma, mb, a);
   }
   return cudaGetLastError();
@@ -422,6 +424,7 @@ cudaError_t gemm_simt(const Batch &A, const Batch &B, int b_trans, int64_t M, in
   if (M % kSB || N % kSB || K % kSK || batch < 1 || batch > 65535) return cudaErrorInvalidValue;
   dim3 grid(static_cast<unsigned>(N / kSB), static_cast<unsigned>(M / kSB), static_cast<unsigned>(batch));
   const float *pa = static_cast<const float *>(A.ptr), *pb = static_cast<const float *>(B.ptr);
+  count_launch();
   if (b_trans)
     gemm_simt_kernel<1><<<grid, 256, 0, stream>>>(pa, pb, K, A.cols, B.cols, A.stride, B.stride, to_epi(ep, M, N));
   else
@@ -431,6 +434,7 @@ cudaError_t gemm_simt(const Batch &A, const Batch &B, int b_trans, int64_t M, in
 
 cudaError_t launch_pack(const PackArgs &a, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(a.parts), static_cast<unsigned>(a.n_tiles));
+  count_launch();
   pack_kernel<<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
@@ -438,6 +442,7 @@ cudaError_t launch_pack(const PackArgs &a, cudaStream_t stream) {
 cudaError_t launch_normalize(const NormArgs &a, cudaStream_t stream) {
   const int64_t chunks = (a.elems + 8191) / 8192;
   dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(a.n_tiles));
+  count_launch();
   normalize_kernel<<<grid, 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
@@ -447,6 +452,7 @@ cudaError_t launch_unpack(const UnpackArgs &a, cudaStream_t stream) {
   const int64_t side = a.n > a.m ? a.n : a.m;   // a tile has at most max(n, m) rows
   const int64_t parts = (side + rpp - 1) / rpp;
   dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(a.n_tiles));
+  count_launch();
   unpack_kernel<<<grid, 256, 0, stream>>>(a, rpp);
   return cudaGetLastError();
 }
@@ -455,12 +461,14 @@ cudaError_t launch_add_identity(const float *z32, float a, float *q32, void *q16
                                 int64_t batch, cudaStream_t stream) {
   const int64_t total = n * n * batch;
   const int blocks = static_cast<int>((total + 255) / 256 < 65535 ? (total + 255) / 256 : 65535);
+  count_launch();
   add_identity_kernel<<<blocks, 256, 0, stream>>>(z32, a, q32, q16, q16_dtype, n, total);
   return cudaGetLastError();
 }
 
 cudaError_t launch_to16(const float *x32, void *x16, int32_t dtype, int64_t count, cudaStream_t stream) {
   const int blocks = static_cast<int>((count + 255) / 256 < 65535 ? (count + 255) / 256 : 65535);
+  count_launch();
   to16_kernel<<<blocks, 256, 0, stream>>>(x32, x16, dtype, count);
   return cudaGetLastError();
 }

@@ -20,7 +20,7 @@ OK = 0
 OP_NS_TILED, OP_NS_FULL, OP_GRAM_NS, OP_MOMENTUM_STEP = 0, 1, 2, 3
 EXPORTS = ("himuon_ns_tiled", "himuon_ns_full", "himuon_gram_ns", "himuon_momentum_step",
            "himuon_workspace_size", "himuon_get_device_status", "himuon_status_string",
-           "himuon_version", "himuon_plan_tiles")
+           "himuon_version", "himuon_plan_tiles", "himuon_launch_count")
 
 
 class Mat(ctypes.Structure):
@@ -70,6 +70,7 @@ def load() -> ctypes.CDLL:
         lib.himuon_status_string.argtypes = [ctypes.c_int]
         lib.himuon_status_string.restype = ctypes.c_char_p
         lib.himuon_version.restype = ctypes.c_int
+        lib.himuon_launch_count.restype = i64
         lib.himuon_plan_tiles.argtypes = [P(Mat), i32, P(Split), i32, P(i64), i64]
         lib.himuon_plan_tiles.restype = i64
         _lib = lib
@@ -200,6 +201,11 @@ def momentum_step(W, M, G, mu: float, lr: float, p: Params, splits=None, update_
                                      _stream(stream))
     _check(rc, "himuon_momentum_step")
     return _ws
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued since it was loaded (host counter)."""
+    return int(load().himuon_launch_count())
 
 
 def device_status(stream=None) -> int:
