@@ -69,7 +69,8 @@ enum {
   HIMUON_ERR_CUDA = -5,         /* a CUDA runtime/driver call failed */
   HIMUON_ERR_TIMEOUT = -6,      /* device: a bounded wait gave up (device status only) */
   HIMUON_ERR_DEVICE = -7,       /* device: inconsistent descriptor seen by a kernel */
-  HIMUON_ERR_NO_DEVICE = -8     /* no usable sm_100 device */
+  HIMUON_ERR_NO_DEVICE = -8,    /* no usable sm_100 device */
+  HIMUON_ERR_TOO_LARGE = -9     /* himuon_ns_static: the call needs more scratch than its fixed array */
 };
 
 /* One row-major matrix in device memory. */
@@ -177,6 +178,38 @@ HIMUON_API const char *himuon_status_string(int code);
 
 /* HIMUON_VERSION of the loaded library. */
 HIMUON_API int himuon_version(void);
+
+/*
+ * Allocation-free variant of the staged (HBM) path of himuon_ns_tiled /
+ * himuon_ns_full.  The paper has no counterpart to this entry point: it serves
+ * callers that cannot allocate device memory themselves -- for instance code
+ * running under a custom allocator or memory pool that owns all of HBM, or a
+ * host runtime that forbids cudaMalloc/cudaFree (which synchronise the device)
+ * during training steps -- and so cannot hand the other entry points a
+ * workspace.
+ *
+ * Arguments are those of himuon_ns_tiled (p->tile <= 0 means full-matrix NS),
+ * minus the workspace.  in/out are still caller buffers.  Every tile, of any
+ * size, runs on the staged path of batched tensor-core GEMMs (or the fp32 path
+ * for compute FP32).  Its scratch -- the tile tables and the chunk workspace --
+ * lives in one file-scope device array of HIMUON_STATIC_SCRATCH_BYTES
+ * (32 MiB) that every GPU which loads the library holds until the process
+ * exits.  The call allocates no device memory (no cudaMalloc, cudaFree or
+ * allocating library routine) and bypasses the plan cache.  A call whose
+ * largest tile (or its tables) does not fit returns HIMUON_ERR_TOO_LARGE
+ * before enqueuing anything; e.g. full-matrix NS fits up to about 1024 x 2048
+ * in bf16 and 1024 x 1024 in fp32.
+ *
+ * The first call on a device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with the device current); make that first call before
+ * any stream capture.  All calls share the one array and it keeps the last
+ * call's contents: calls that overlap on the GPU (on different streams, or
+ * from different host threads) race on it and must be serialised by the
+ * caller.  Calls on one stream are ordered and safe.
+ */
+#define HIMUON_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+HIMUON_API int himuon_ns_static(const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,
+                                const himuon_ns_params *p, void *stream);
 
 /*
  * Number of CUDA kernels this library has enqueued since it was loaded, on all

@@ -719,6 +719,101 @@ int dispatch(int op, const CallMats &cm, const himuon_split *splits, const himuo
 }
 
 }  // namespace
+
+// Staged NS (in -> out) with every device byte it needs taken from one
+// caller-supplied region `scratch` of `scratch_bytes` (256-byte aligned): the
+// block and tile tables first, the per-chunk workspace after them.  Builds the
+// plan on the host and uploads the tables with cudaMemcpyAsync on `stream`;
+// allocates no device memory and does not touch the plan cache.
+int run_staged_into(int op, const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,
+                    const himuon_ns_params *p, void *scratch, size_t scratch_bytes, cudaStream_t stream) {
+  if (!in || !out || !p || !scratch) return HIMUON_ERR_INVALID;
+  if (op != HIMUON_OP_NS_TILED && op != HIMUON_OP_NS_FULL) return HIMUON_ERR_INVALID;
+  int rc = check_params(p);
+  if (rc) return rc;
+  CallMats cm;
+  cm.n = n;
+  cm.role[kRoleIn] = in;
+  cm.role[kRoleOut] = out;
+  rc = check_call(cm, splits);
+  if (rc) return rc;
+  rc = check_device();
+  if (rc) return rc;
+  Plan plan;
+  cudaGetDevice(&plan.device);
+  rc = make_blocks(cm, splits, op == HIMUON_OP_NS_FULL || p->tile <= 0 ? 0 : p->tile, plan.blocks, &plan.n_tiles);
+  if (rc) return rc;
+  std::vector<DevBlock> dblocks(plan.blocks.size());
+  for (size_t bi = 0; bi < plan.blocks.size(); ++bi) {
+    const HostBlock &b = plan.blocks[bi];
+    DevBlock &d = dblocks[bi];
+    memset(&d, 0, sizeof d);
+    d.tile_begin = b.tile_begin;
+    d.tiles_r = static_cast<int32_t>(b.tiles_r);
+    d.tiles_c = static_cast<int32_t>(b.tiles_c);
+    d.rows = static_cast<int32_t>(b.rows);
+    d.cols = static_cast<int32_t>(b.cols);
+    d.T = static_cast<int32_t>(b.T);
+    d.mat = b.mat;
+    for (int r = 0; r < kNumRoles; ++r) {
+      d.tmap[r] = -1;
+      if (!cm.role[r]) continue;
+      const himuon_mat &m = cm.role[r][b.mat];
+      d.ptr[r] = block_ptr(m, b);
+      d.ld[r] = m.ld;
+      d.dtype[r] = m.dtype;
+    }
+  }
+  std::map<std::pair<int64_t, int64_t>, size_t> cls;
+  for (size_t bi = 0; bi < plan.blocks.size(); ++bi) {
+    const HostBlock &b = plan.blocks[bi];
+    for (int64_t tr = 0; tr < b.tiles_r; ++tr)
+      for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
+        DevTile t;
+        t.block = static_cast<int32_t>(bi);
+        t.r0 = static_cast<int32_t>(tr * b.T);
+        t.c0 = static_cast<int32_t>(tc * b.T);
+        t.h = static_cast<int32_t>(std::min(b.T, b.rows - t.r0));
+        t.w = static_cast<int32_t>(std::min(b.T, b.cols - t.c0));
+        t.transposed = t.h > t.w ? 1 : 0;
+        const int64_t nn = round_up(std::min(t.h, t.w), 128), mm = round_up(std::max(t.h, t.w), 128);
+        auto it = cls.find({nn, mm});
+        if (it == cls.end()) {
+          it = cls.emplace(std::make_pair(nn, mm), plan.classes.size()).first;
+          TileClass c;
+          c.n = nn;
+          c.m = mm;
+          c.padded = false;
+          plan.classes.push_back(c);
+        }
+        TileClass &c = plan.classes[it->second];
+        if (std::min(t.h, t.w) != nn || std::max(t.h, t.w) != mm) c.padded = true;
+        c.tiles.push_back(t);
+      }
+  }
+  std::vector<DevTile> dtiles;
+  for (TileClass &c : plan.classes) {
+    c.dev_offset = static_cast<int64_t>(dtiles.size());
+    dtiles.insert(dtiles.end(), c.tiles.begin(), c.tiles.end());
+  }
+  const size_t sb = round_up(sizeof(DevBlock) * dblocks.size(), 256);
+  const size_t st = round_up(sizeof(DevTile) * dtiles.size(), 256);
+  if (sb + st >= scratch_bytes) return HIMUON_ERR_TOO_LARGE;
+  const size_t ws_bytes = scratch_bytes - sb - st;
+  if (static_cast<int64_t>(ws_bytes) < staged_ws_bytes(plan, p->compute, false)) return HIMUON_ERR_TOO_LARGE;
+  char *base = static_cast<char *>(scratch);
+  if (cudaMemcpyAsync(base, dblocks.data(), sizeof(DevBlock) * dblocks.size(), cudaMemcpyHostToDevice, stream) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(base + sb, dtiles.data(), sizeof(DevTile) * dtiles.size(), cudaMemcpyHostToDevice, stream) !=
+          cudaSuccess)
+    return HIMUON_ERR_CUDA;
+  plan.d_blocks = reinterpret_cast<DevBlock *>(base);
+  plan.d_tiles = reinterpret_cast<DevTile *>(base + sb);
+  himuon_ns_params q = *p;
+  q.chunk_bytes = 0;
+  return run_staged(plan, op, q, 0.f, 0.f, base + sb + st, ws_bytes, stream);
+}
+
 }  // namespace himuon
 
 using namespace himuon;
@@ -835,6 +930,7 @@ const char *himuon_status_string(int code) {
     case HIMUON_ERR_TIMEOUT: return "device wait timed out";
     case HIMUON_ERR_DEVICE: return "inconsistent descriptor seen on the device";
     case HIMUON_ERR_NO_DEVICE: return "no usable sm_100 device";
+    case HIMUON_ERR_TOO_LARGE: return "problem needs more scratch than himuon_ns_static's fixed device array";
     default: return "unknown status";
   }
 }

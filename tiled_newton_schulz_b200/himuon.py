@@ -20,7 +20,9 @@ OK = 0
 OP_NS_TILED, OP_NS_FULL, OP_GRAM_NS, OP_MOMENTUM_STEP = 0, 1, 2, 3
 EXPORTS = ("himuon_ns_tiled", "himuon_ns_full", "himuon_gram_ns", "himuon_momentum_step",
            "himuon_workspace_size", "himuon_get_device_status", "himuon_status_string",
-           "himuon_version", "himuon_plan_tiles", "himuon_launch_count")
+           "himuon_version", "himuon_plan_tiles", "himuon_launch_count", "himuon_ns_static")
+ERR_TOO_LARGE = -9
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 class Mat(ctypes.Structure):
@@ -60,6 +62,8 @@ def load() -> ctypes.CDLL:
         for name in ("himuon_ns_tiled", "himuon_ns_full", "himuon_gram_ns"):
             getattr(lib, name).argtypes = ns_sig
             getattr(lib, name).restype = ctypes.c_int
+        lib.himuon_ns_static.argtypes = [P(Mat), P(Mat), i32, P(Split), P(Params), vp]
+        lib.himuon_ns_static.restype = ctypes.c_int
         lib.himuon_momentum_step.argtypes = [P(Mat), P(Mat), P(Mat), i32, ctypes.c_float, ctypes.c_float, P(Split),
                                              P(Params), P(Mat), vp, ctypes.c_size_t, vp]
         lib.himuon_momentum_step.restype = ctypes.c_int
@@ -186,6 +190,20 @@ def ns_full(inputs, outputs, p: Params, splits=None, workspace=None, stream=None
 
 def gram_ns(inputs, outputs, p: Params, splits=None, workspace=None, stream=None):
     return _ns_call("himuon_gram_ns", OP_GRAM_NS, inputs, outputs, p, splits, workspace, stream)
+
+
+def ns_static(inputs, outputs, p: Params, splits=None, stream=None) -> int:
+    """Staged NS with the library's own fixed device scratch (no workspace).
+
+    For callers that cannot allocate device memory; returns the status code
+    (ERR_TOO_LARGE when the call does not fit the 32 MiB array) instead of
+    raising, so callers can fall back.
+    """
+    if len(inputs) != len(outputs):
+        raise ValueError("inputs and outputs differ in length")
+    mi, mo = _mats(inputs), _mats(outputs)
+    sp, _keep = _splits(splits, len(inputs))
+    return int(load().himuon_ns_static(mi, mo, len(inputs), sp, ctypes.byref(p), _stream(stream)))
 
 
 def momentum_step(W, M, G, mu: float, lr: float, p: Params, splits=None, update_out=None, workspace=None,
