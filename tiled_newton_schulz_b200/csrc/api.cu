@@ -687,6 +687,11 @@ int run_resident(const Plan &plan, int op, const himuon_ns_params &p, float mu, 
   a.eps = p.eps;
   a.safety = p.safety > 0.f ? p.safety : 1.f;
   a.status = status_ptr();
+  // the kernel keeps a compact copy of the block table in shared memory when
+  // it fits: 32-bit tile numbers, 16-bit tile counts and tensor-map indices
+  bool fits = static_cast<int>(plan.blocks.size()) <= resident_max_smem_blocks() && plan.n_tiles < (int64_t(1) << 31);
+  for (const HostBlock &b : plan.blocks) fits = fits && b.tiles_c < 65536 && b.cols < (int64_t(1) << 31);
+  a.smem_blocks = fits ? 1 : 0;
   make_resident_steps(a, p.coeffs, p.steps);
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, plan.device);

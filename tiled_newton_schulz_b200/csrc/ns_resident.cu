@@ -7,21 +7,33 @@
 // zero border stays zero through X X^T, A^2 and B X and leaves ||X||_F alone;
 // and the transpose of a tall tile is not needed because NS(X^T) = NS(X)^T).
 //
-// One persistent CTA per SM runs two independent tile "groups" of 4 warps each
-// plus one MMA-issuing warp, so that one group's tcgen05 MMAs overlap the other
-// group's TMEM -> register -> shared-memory conversions.  Per group:
+// One persistent CTA per SM runs two independent tile "groups" of 8 warps
+// (two per TMEM lane quarter, each owning 64 of a row's 128 columns), so that
+// one group's tcgen05 MMAs overlap the other group's TMEM -> register ->
+// shared-memory conversions.  Each group issues its own MMAs from one thread
+// right after a group-wide named barrier (no hand-off to a separate MMA warp);
+// that thread's tcgen05.commit tracks exactly its group's MMAs.  Per group:
 //   shared memory  X_s (16-bit iterate operand, 32 KB), S_s (16-bit operand, 32 KB), W_s (32 KB)
-//   tensor memory  D_P (128 cols fp32: A, then B / b), D_X (128 cols fp32 iterate)
-// Per step the group runs three 128x128x128 MMAs:
-//   MMA1  D_P  = X X^T                               (X_s twice, K-major)
-//   MMA2  D_P += sign(c/b) S S^T,  S = r(sqrt|c/b| A)    -> D_P = A + (c/b) A^2 = B / b
-//   MMA3  D_X += Bop X,  Bop = r(b D_P + (a - 1) I)      (X_s read MN-major)
+//   tensor memory  D_P (128 cols fp32: A, then B / b), D_X (128 cols fp32: the iterate)
+// Per step the group runs three 128x128x128 MMAs, every A operand read from
+// TMEM and every B operand from shared memory:
+//   MMA1  D_P  = X X^T                          A: X (packed in D_X),   B: X_s (K-major)
+//   MMA2  D_P += sign(c/b) S S^T                A: S (packed in D_X),   B: S_s,  S = r(sqrt|c/b| A)
+//                                               -> D_P = A + (c/b) A^2 = B / b
+//   MMA3  D_X  = Bop X,  Bop = r(b D_P + a I)   A: Bop (packed in D_P), B: X_s (MN-major)
 // r() rounds to the 16-bit operand type (fp16 or bf16, chosen per call).
-// D_X holds the fp32 iterate X_t itself, so MMA3 realises X <- a X + B X as
-// X + ((a - 1) I + B) X: the fp32 part is carried exactly and only the
-// correction goes through 16-bit operands.  The momentum update M' = mu M + G
-// is fused into the prologue (M' written back once) and W <- W - lr O into the
-// epilogue, so HBM sees one read and one write per element and role.
+// MMA3 forms the whole update X <- a X + B X = (a I + B) X with fp32
+// accumulation.  A 16-bit operand is packed two per 32-bit TMEM column in
+// place: each thread, having read its 64 fp32 columns of a region, writes
+// their 16-bit values to the first 32 of those columns (nobody else reads
+// them), or into D_X while D_X holds nothing live.  Keeping A operands out of
+// shared memory halves the operand traffic there (N = 128 MMAs with both
+// operands in shared memory run at the shared-memory bandwidth limit).
+// The momentum update M' = mu M + G is fused into the prologue (M' written
+// back once) and W <- W - lr O into the epilogue, so HBM sees one read and one
+// write per element and role.  The next tile's inputs are loaded (TMA) as soon
+// as this tile's last MMA has released X_s / S_s, under the final epilogue; W
+// lands in its own buffer.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -34,25 +46,50 @@ namespace himuon {
 
 namespace {
 
-constexpr int kGroupThreads = 128;
-constexpr int kMmaWarp = 8;
-constexpr int kThreads = 9 * 32;
+constexpr int kGroupWarps = 8;
+constexpr int kGroupThreads = kGroupWarps * 32;
+constexpr int kThreads = 2 * kGroupThreads;
 constexpr uint32_t kHalf = 16384;          // one 64-column, 128-row swizzled half tile
 constexpr uint32_t kOffX = 0, kOffS = 32768, kOffW = 65536, kGroupBytes = 98304;
 constexpr uint32_t kOffBars = 2 * kGroupBytes;
-constexpr uint32_t kSmemBytes = kOffBars + 256 + 1024;   // + alignment slack
+constexpr int kMaxSmemBlocks = 256;        // block tables up to this size live in shared memory
+constexpr uint32_t kOffBlocks = kOffBars + 512;
+constexpr uint32_t kSmemBytes = kOffBlocks + kMaxSmemBlocks * 24 + 1024;   // + alignment slack
+
+struct TileCoord {
+  int32_t blk;       // -1: no tile
+  int32_t x0, y0, cols;
+  int32_t tm[kNumRoles];
+};
+
+// What the tile decoder needs of a DevBlock, kept in shared memory (used when
+// the host found that the block table fits: ResidentArgs::smem_blocks).
+struct SBlock {
+  int32_t tile_begin;
+  int32_t cols;
+  uint16_t tiles_c, T;
+  int16_t tm[kNumRoles];
+  int32_t pad;
+};
+static_assert(sizeof(SBlock) == 24, "SBlock layout");
 
 struct Smem {
   uint8_t *base;
   __device__ uint8_t *x(int g) const { return base + g * kGroupBytes + kOffX; }
   __device__ uint8_t *s(int g) const { return base + g * kGroupBytes + kOffS; }
   __device__ uint8_t *w(int g) const { return base + g * kGroupBytes + kOffW; }
-  __device__ uint64_t *bar_ld(int g) const { return reinterpret_cast<uint64_t *>(base + kOffBars) + 3 * g + 0; }
-  __device__ uint64_t *bar_mma(int g) const { return reinterpret_cast<uint64_t *>(base + kOffBars) + 3 * g + 1; }
-  __device__ uint64_t *bar_epi(int g) const { return reinterpret_cast<uint64_t *>(base + kOffBars) + 3 * g + 2; }
-  __device__ float *red(int g) const { return reinterpret_cast<float *>(base + kOffBars + 64) + 4 * g; }
+  __device__ uint64_t *bar(int g, int i) const { return reinterpret_cast<uint64_t *>(base + kOffBars) + 4 * g + i; }
+  __device__ uint64_t *bar_ld(int g) const { return bar(g, 0); }    // M (or input) and G landed
+  __device__ uint64_t *bar_w(int g) const { return bar(g, 1); }     // W landed
+  __device__ uint64_t *bar_mma(int g) const { return bar(g, 2); }   // the group's MMA job finished
+  __device__ float *red(int g) const { return reinterpret_cast<float *>(base + kOffBars + 64) + kGroupWarps * g; }
   __device__ uint32_t *tmem_slot() const { return reinterpret_cast<uint32_t *>(base + kOffBars + 128); }
   __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(base + kOffBars + 132); }
+  __device__ SBlock *blocks() const { return reinterpret_cast<SBlock *>(base + kOffBlocks); }
+  // current / next tile coordinates of group g (read and written by its issuing thread only)
+  __device__ TileCoord *coord(int g, int i) const {
+    return reinterpret_cast<TileCoord *>(base + kOffBars + 256) + 2 * g + i;
+  }
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, const Smem &sm, int *status) {
@@ -80,92 +117,122 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
     f[2 * i + 1] = t.y;
   }
 }
-__device__ __forceinline__ uint4 pack8_bf16(const float *f) {
-  uint4 u;
-  __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-  return u;
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
 }
-// 16-bit operand of format F (0: fp16, 1: bf16)
+// two values as a 16-bit operand pair of format F (0: fp16, 1: bf16)
+template <int F>
+__device__ __forceinline__ uint32_t pack2_op(float a, float b) {
+  if (F == 1) return pack2_bf16(a, b);
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ uint4 pack8_bf16(const float *f) {
+  return make_uint4(pack2_bf16(f[0], f[1]), pack2_bf16(f[2], f[3]), pack2_bf16(f[4], f[5]), pack2_bf16(f[6], f[7]));
+}
 template <int F>
 __device__ __forceinline__ uint4 pack8_op(const float *f) {
-  if (F == 1) return pack8_bf16(f);
-  uint4 u;
-  __half2 *h = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
-  return u;
+  return make_uint4(pack2_op<F>(f[0], f[1]), pack2_op<F>(f[2], f[3]), pack2_op<F>(f[4], f[5]),
+                    pack2_op<F>(f[6], f[7]));
 }
 
-// byte offset of 16-byte chunk cg (0..15, i.e. columns 8cg..8cg+7) of row r in
-// a 128x128 bf16 tile stored as two 128B-swizzled 64-column halves.
-__device__ __forceinline__ uint32_t chunk_off(uint32_t r, uint32_t cg) {
-  return (cg >> 3) * kHalf + sw128_off(r, cg & 7u);
-}
-
-// Row r of a 128-column fp32 TMEM region -> scale * v (+ diag on column r) as
-// 16-bit operands in the swizzled tile.  With WB the scaled fp32 values are
-// also written back to the TMEM region.
-template <int F, bool DIAG, bool WB>
-__device__ __forceinline__ void tmem_row_to_op(uint32_t taddr, uint8_t *dst, uint32_t r, float scale, float diag) {
-  const uint32_t q = r >> 5, ln = r & 31u;
+// This thread's 64 columns (half `hf`) of row r of the 128-column fp32 TMEM
+// region at `src` -> r(scale * v), written twice: to the swizzled shared tile
+// (B operand) and packed to TMEM columns [64 hf, 64 hf + 32) of the region at
+// `pk` (A operand).  `pk` may equal `src`: the thread reads all 64 columns
+// before it writes the first 32.
+template <int F, bool SCALE>
+__device__ __forceinline__ void tmem_row_to_op(uint32_t src, uint32_t pk, uint8_t *dst, uint32_t r, uint32_t hf,
+                                               float scale) {
+  // 32 columns at a time keeps the live register set small (no spills)
+  uint8_t *row = dst + hf * kHalf;
+  const uint32_t c0 = 64u * hf;
 #pragma unroll
-  for (int i = 0; i < 4; i += 2) {
-    float v0[32], v1[32];
-    tmem_ld32(taddr + 32 * i, v0);
-    tmem_ld32(taddr + 32 * (i + 1), v1);
+  for (int i = 0; i < 2; ++i) {
+    float v[32];
+    tmem_ld32(src + c0 + 32 * i, v);
     tmem_wait_ld();
+    uint32_t p[16];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      v0[e] *= scale;
-      v1[e] *= scale;
-    }
-    if (DIAG) {
-      if (q == static_cast<uint32_t>(i)) {
+    for (int e = 0; e < 16; ++e)
+      p[e] = SCALE ? pack2_op<F>(v[2 * e] * scale, v[2 * e + 1] * scale) : pack2_op<F>(v[2 * e], v[2 * e + 1]);
+    tmem_st16(pk + c0 + 16 * i, p);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v0[e] += (static_cast<uint32_t>(e) == ln) ? diag : 0.f;
-      } else if (q == static_cast<uint32_t>(i + 1)) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v1[e] += (static_cast<uint32_t>(e) == ln) ? diag : 0.f;
-      }
-    }
-    if (WB) {
-      tmem_st32(taddr + 32 * i, v0);
-      tmem_st32(taddr + 32 * (i + 1), v1);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      *reinterpret_cast<uint4 *>(dst + chunk_off(r, 4 * i + j)) = pack8_op<F>(v0 + 8 * j);
-      *reinterpret_cast<uint4 *>(dst + chunk_off(r, 4 * (i + 1) + j)) = pack8_op<F>(v1 + 8 * j);
-    }
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4 *>(row + sw128_off(r, 4 * i + j)) = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
   }
-  if (WB) tmem_wait_st();
+  tmem_wait_st();
 }
 
-__device__ __forceinline__ void signal_mma(uint64_t *bar) {
-  fence_proxy_async_smem();
-  tc_fence_before();
-  mbar_arrive(bar);
+// Bop = r(beta * D_P + diag * I) for this thread's 64 columns of row r,
+// packed two per 32-bit word into TMEM columns [64 hf, 64 hf + 32) of D_P
+// (columns this thread has already read; nobody else reads them).
+template <int F>
+__device__ __forceinline__ void tmem_row_to_tmem_op(uint32_t taddr, uint32_t r, uint32_t hf, float beta, float diag) {
+  const uint32_t c0 = 64u * hf;
+  const bool mine = (r >> 6) == hf;            // the diagonal element sits in this thread's columns
+  const uint32_t dl = (r & 63u);               // its position among them
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float v[32];
+    tmem_ld32(taddr + c0 + 32 * i, v);
+    tmem_wait_ld();
+    uint32_t p[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t k = 32u * i + 2u * e;
+      const float a0 = fmaf(beta, v[2 * e], (mine && dl == k) ? diag : 0.f);
+      const float a1 = fmaf(beta, v[2 * e + 1], (mine && dl == k + 1) ? diag : 0.f);
+      p[e] = pack2_op<F>(a0, a1);
+    }
+    tmem_st16(taddr + c0 + 16 * i, p);   // columns [c0, c0 + 32) were read before any is written
+  }
+  tmem_wait_st();
 }
 
-struct TileCoord {
-  const DevBlock *blk;
-  int32_t x0, y0;
-};
+__device__ __forceinline__ bool use_smem_blocks(const ResidentArgs &a) {
+  return a.smem_blocks != 0 && a.n_blocks <= kMaxSmemBlocks;
+}
 
-__device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, int64_t tile) {
+// Block of `tile` by binary search over tile_begin, in the shared-memory copy
+// of the block table when it fits there (a few shared loads), else in global.
+__device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, const Smem &sm, int64_t tile) {
+  TileCoord t;
+  t.blk = -1;
+  t.x0 = t.y0 = t.cols = 0;
+#pragma unroll
+  for (int r = 0; r < kNumRoles; ++r) t.tm[r] = -1;
+  if (tile >= a.n_tiles) return t;
   int lo = 0, hi = a.n_blocks - 1;
-  while (lo < hi) {  // last block with tile_begin <= tile
+  if (use_smem_blocks(a)) {
+    const SBlock *sb = sm.blocks();
+    while (lo < hi) {  // last block with tile_begin <= tile
+      const int mid = (lo + hi + 1) >> 1;
+      if (sb[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
+    }
+    const SBlock &b = sb[lo];
+    const int32_t local = static_cast<int32_t>(tile) - b.tile_begin;
+    t.blk = lo;
+    t.y0 = (local / b.tiles_c) * b.T;
+    t.x0 = (local % b.tiles_c) * b.T;
+    t.cols = b.cols;
+#pragma unroll
+    for (int r = 0; r < kNumRoles; ++r) t.tm[r] = b.tm[r];
+    return t;
+  }
+  while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (a.blocks[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
   }
-  const DevBlock *b = a.blocks + lo;
-  const int64_t local = tile - b->tile_begin;
-  TileCoord t;
-  t.blk = b;
-  t.y0 = static_cast<int32_t>(local / b->tiles_c) * b->T;
-  t.x0 = static_cast<int32_t>(local % b->tiles_c) * b->T;
+  const DevBlock &b = a.blocks[lo];
+  const int64_t local = tile - b.tile_begin;
+  t.blk = lo;
+  t.y0 = static_cast<int32_t>(local / b.tiles_c) * b.T;
+  t.x0 = static_cast<int32_t>(local % b.tiles_c) * b.T;
+  t.cols = b.cols;
+#pragma unroll
+  for (int r = 0; r < kNumRoles; ++r) t.tm[r] = b.tmap[r];
   return t;
 }
 
@@ -183,56 +250,119 @@ __device__ __forceinline__ void prefetch_tile(const CUtensorMap *m, int32_t x0, 
   if (x0 + 64 < cols) tma_prefetch_l2_2d(m, x0 + 64, y0);
 }
 
-// ------------------------------------------------------------------ epilogue group
+// M (or the NS input) -> X_s and, for a momentum step, G -> S_s.
+__device__ __forceinline__ void issue_mg(const ResidentArgs &a, const Smem &sm, int g, const TileCoord &t) {
+  const bool step_mode = a.mode == 1;
+  mbar_arrive_expect_tx(sm.bar_ld(g), step_mode ? 4 * kHalf : 2 * kHalf);
+  load_tile(a.tmaps + t.tm[kRoleIn], sm.x(g), t.x0, t.y0, sm.bar_ld(g));
+  if (step_mode) load_tile(a.tmaps + t.tm[kRoleG], sm.s(g), t.x0, t.y0, sm.bar_ld(g));
+}
+__device__ __forceinline__ void issue_w(const ResidentArgs &a, const Smem &sm, int g, const TileCoord &t) {
+  mbar_arrive_expect_tx(sm.bar_w(g), 2 * kHalf);
+  load_tile(a.tmaps + t.tm[kRoleW], sm.w(g), t.x0, t.y0, sm.bar_w(g));
+}
+
+// ------------------------------------------------------------------ MMA issue
+// Shared-memory descriptors differ only in the start-address field (bits
+// 0..13, address >> 4; every address here is below 256 KB), so each one is a
+// fixed template plus a per-operand address and a compile-time offset.
+//   K-major operand (X_s, S_s): 128 rows x 128 16-bit values, two swizzled
+//   64-column halves; k-step kk covers columns 16kk..16kk+15.
+//   MN-major view of X_s (its rows are K): k-step kk covers rows 16kk..16kk+15,
+//   the two 64-column halves are kHalf apart.
+__device__ __forceinline__ uint64_t desc_k(uint64_t tmpl, uint32_t base4, int kk) {
+  return tmpl + base4 + static_cast<uint32_t>(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+}
+__device__ __forceinline__ uint64_t desc_mn(uint64_t tmpl, uint32_t base4, int kk) {
+  return tmpl + base4 + static_cast<uint32_t>((kk * 2048) >> 4);
+}
+
+enum Job { kJobGram = 0, kJobSquare = 1, kJobUpdate = 2 };
+
+// All threads of the group have written (and fenced) the operands of `job`:
+// one thread issues its eight 128x128x16 MMAs and commits them to bar_mma.
+template <int F, int JOB>
+__device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st);
+
+template <int F, int JOB>
+__device__ __forceinline__ void group_issue(const ResidentArgs &a, const Smem &sm, int g, int gt, uint32_t dP,
+                                            const ResidentStep *st) {
+  named_bar_sync(1 + g, kGroupThreads);
+  if (gt >= 32) return;
+  // Lanes 1..31 of the issuing warp wait here for lane 0: if they went on to
+  // spin on the completion barrier, the warp would interleave their
+  // (suspending) try_wait with lane 0's issue and delay the MMAs.
+  if (gt == 0) group_issue_mmas<F, JOB>(sm, g, dP, st);
+  __syncwarp();
+}
+
+template <int F, int JOB>
+__device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st) {
+  tc_fence_after();
+  const uint64_t tk = sw128_desc(0, 16, 1024);
+  const uint32_t dX = dP + 128u;
+  // packed A operand: K columns 0..63 at region + [0, 32), 64..127 at region + [64, 96)
+  if (JOB == kJobGram) {
+    const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
+    constexpr uint32_t id = idesc_f16(128, 128, F, 0, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) mma_ts(dP, dX + (kk >> 2) * 64 + (kk & 3) * 8, desc_k(tk, x4, kk), id, kk > 0);
+  } else if (JOB == kJobSquare) {
+    const uint32_t s4 = smem_u32(sm.s(g)) >> 4;
+    const uint32_t id = idesc_f16(128, 128, F, 0, 0, st->neg2);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ts(dP, dX + (kk >> 2) * 64 + (kk & 3) * 8, desc_k(tk, s4, kk), id, st->acc2 | (kk > 0));
+  } else {
+    const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
+    const uint64_t tmn = sw128_desc(0, kHalf, 1024);
+    constexpr uint32_t id = idesc_f16(128, 128, F, 0, 1, 0);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) mma_ts(dX, dP + (kk >> 2) * 64 + (kk & 3) * 8, desc_mn(tmn, x4, kk), id, kk > 0);
+  }
+  mma_commit(sm.bar_mma(g));
+}
+
+// ------------------------------------------------------------------ one tile group
 template <int F>
 __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem, int g) {
-  const int gt = threadIdx.x - g * kGroupThreads;   // 0..127 == tile row
+  const int gt = threadIdx.x - g * kGroupThreads;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t r = static_cast<uint32_t>(gt);
-  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t tP = tmem + lane_base + 256u * g;     // D_P
-  const uint32_t tX = tP + 128u;                       // D_X
+  const int wig = warp - g * kGroupWarps;              // warp in group, 0..7
+  const uint32_t q = static_cast<uint32_t>(warp & 3);  // TMEM lane quarter
+  const uint32_t hf = static_cast<uint32_t>(wig >> 2); // column half owned by this thread
+  const uint32_t r = q * 32 + lane;                    // tile row
+  const uint32_t dP = tmem + 256u * g;                 // D_P (lane 0); D_X = dP + 128
+  const uint32_t tP = dP + ((q * 32) << 16);           // this warp's lanes of D_P
+  const uint32_t tX = tP + 128u;                       // ... and of D_X
   uint8_t *Xs = sm.x(g), *Ss = sm.s(g), *Ws = sm.w(g);
   const int bar_id = 1 + g;
   const bool step_mode = a.mode == 1;
+  const bool has_w = step_mode && a.has_w;
   const int64_t grid = gridDim.x;
   uint32_t it = 0, job = 0;
+  bool mg_issued = false;   // (issuing thread) this tile's M/G loads went out during the previous tile
+  TileCoord *cur = sm.coord(g, 0), *nxt = sm.coord(g, 1);
+  if (gt == 0) *cur = decode_tile(a, sm, blockIdx.x + g * grid);
 
   for (int64_t tile = blockIdx.x + g * grid; tile < a.n_tiles; tile += 2 * grid, ++it) {
-    const TileCoord tc = decode_tile(a, tile);
-    const DevBlock &b = *tc.blk;
-    const CUtensorMap *mIn = a.tmaps + b.tmap[kRoleIn];
     if (gt == 0) {
-      bulk_wait_read0();  // the previous tile's stores have finished reading X_s / W_s
-      uint32_t bytes = 2 * kHalf;
-      if (step_mode) bytes += 2 * kHalf + (a.has_w ? 2 * kHalf : 0);
-      mbar_arrive_expect_tx(sm.bar_ld(g), bytes);
-      load_tile(mIn, Xs, tc.x0, tc.y0, sm.bar_ld(g));
-      if (step_mode) {
-        load_tile(a.tmaps + b.tmap[kRoleG], Ss, tc.x0, tc.y0, sm.bar_ld(g));
-        if (a.has_w) load_tile(a.tmaps + b.tmap[kRoleW], Ws, tc.x0, tc.y0, sm.bar_ld(g));
-      }
-      const int64_t nxt = tile + 2 * grid;
-      if (nxt < a.n_tiles) {  // warm L2 with this group's next tile
-        const TileCoord nc = decode_tile(a, nxt);
-        const DevBlock &nb = *nc.blk;
-        prefetch_tile(a.tmaps + nb.tmap[kRoleIn], nc.x0, nc.y0, nb.cols);
-        if (step_mode) {
-          prefetch_tile(a.tmaps + nb.tmap[kRoleG], nc.x0, nc.y0, nb.cols);
-          if (a.has_w) prefetch_tile(a.tmaps + nb.tmap[kRoleW], nc.x0, nc.y0, nb.cols);
-        }
-      }
+      bulk_wait_read0();  // the previous tile's stores have finished reading S_s / W_s
+      if (!mg_issued) issue_mg(a, sm, g, *cur);
+      if (has_w) issue_w(a, sm, g, *cur);
     }
+    __syncwarp();
     if (!wait_or_abort(sm.bar_ld(g), it & 1u, sm, a.status)) break;
 
-    // ---- prologue: M' = mu M + G (or the plain input), ||.||_F, fp32 copy to D_X
+    // ---- prologue: M' = mu M + G (or the plain input), ||.||_F, fp32 copy to D_X.
+    // M' (bf16, for the write-back) replaces G in S_s, so X_s is free for X_0 at once.
     float sumsq = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       float v[32];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t off = chunk_off(r, 4 * i + j);
+        const uint32_t off = hf * kHalf + sw128_off(r, 4 * i + j);
         float m[8];
         unpack8(*reinterpret_cast<const uint4 *>(Xs + off), m);
         if (step_mode) {
@@ -240,7 +370,7 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
           unpack8(*reinterpret_cast<const uint4 *>(Ss + off), gg);
 #pragma unroll
           for (int e = 0; e < 8; ++e) m[e] = fmaf(a.mu, m[e], gg[e]);
-          *reinterpret_cast<uint4 *>(Xs + off) = pack8_bf16(m);
+          *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(m);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -248,67 +378,92 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
           sumsq = fmaf(m[e], m[e], sumsq);
         }
       }
-      tmem_st32(tX + 32 * i, v);
+      tmem_st32(tX + 64 * hf + 32 * i, v);
     }
     tmem_wait_st();
-    if (step_mode) {
-      fence_proxy_async_smem();
-      named_bar_sync(bar_id, kGroupThreads);
-      if (gt == 0) {
-        store_tile(mIn, Xs, tc.x0, tc.y0, b.cols);
-        bulk_commit();
+    sumsq = warp_sum(sumsq);
+    if (lane == 0) sm.red(g)[wig] = sumsq;
+    if (step_mode) fence_proxy_async_smem();
+    named_bar_sync(bar_id, kGroupThreads);   // M' complete in S_s, partial sums visible, M read
+    if (step_mode && gt == 0) {
+      store_tile(a.tmaps + cur->tm[kRoleIn], Ss, cur->x0, cur->y0, cur->cols);
+      bulk_commit();
+    }
+    __syncwarp();
+    float total = 0.f;
+#pragma unroll
+    for (int i = 0; i < kGroupWarps; ++i) total += sm.red(g)[i];
+    const float rho = (sqrtf(total) + a.eps) * a.safety;
+
+    // ---- X_0 = r(M' / rho) to X_s and (packed) to D_X
+    tmem_row_to_op<F, true>(tX, tX, Xs, r, hf, 1.0f / rho);
+    // M' must have left S_s before the first conversion overwrites it; that
+    // conversion follows MMA1, which the issuing thread starts only after this.
+    if (step_mode && gt == 0) bulk_wait_read0();
+    __syncwarp();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr);
+
+    if (gt == 0) {   // next tile of this group, while MMA1 runs
+      *nxt = decode_tile(a, sm, tile + 2 * grid);
+      if (nxt->blk >= 0) {
+        prefetch_tile(a.tmaps + nxt->tm[kRoleIn], nxt->x0, nxt->y0, nxt->cols);
+        if (step_mode) prefetch_tile(a.tmaps + nxt->tm[kRoleG], nxt->x0, nxt->y0, nxt->cols);
+        if (has_w) prefetch_tile(a.tmaps + nxt->tm[kRoleW], nxt->x0, nxt->y0, nxt->cols);
       }
     }
-    sumsq = warp_sum(sumsq);
-    if (lane == 0) sm.red(g)[warp & 3] = sumsq;
-    named_bar_sync(bar_id, kGroupThreads);
-    const float total = sm.red(g)[0] + sm.red(g)[1] + sm.red(g)[2] + sm.red(g)[3];
-    const float rho = (sqrtf(total) + a.eps) * a.safety;
-    const float inv_rho = 1.0f / rho;
-    if (step_mode && gt == 0) bulk_wait_read0();   // M' has left X_s
-    named_bar_sync(bar_id, kGroupThreads);
-
-    // ---- X_0 = M' / rho: operand copy to X_s, fp32 copy back to D_X
-    tmem_row_to_op<F, false, true>(tX, Xs, r, inv_rho, 0.f);
-    signal_mma(sm.bar_epi(g));
+    __syncwarp();
 
     bool ok = true;
     for (int t = 0; t < a.K && ok; ++t) {
-      const ResidentStep &st = a.step[t];
-      // after MMA1: S = r(s A)
+      const ResidentStep *st = &a.step[t];
+      // after MMA1: S = r(s A) to S_s and (packed) to D_X
       if (!(ok = wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status))) break;
       tc_fence_after();
-      tmem_row_to_op<F, false, false>(tP, Ss, r, st.s, 0.f);
-      signal_mma(sm.bar_epi(g));
-      // after MMA2: Bop = r(beta D_P + (a - 1) I)
+      tmem_row_to_op<F, true>(tP, tX, Ss, r, hf, st->s);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      group_issue<F, kJobSquare>(a, sm, g, gt, dP, st);
+      // after MMA2: Bop = r(beta D_P + a I), packed in D_P
       if (!(ok = wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status))) break;
       tc_fence_after();
-      tmem_row_to_op<F, true, false>(tP, Ss, r, st.beta, st.am1);
-      signal_mma(sm.bar_epi(g));
+      tmem_row_to_tmem_op<F>(tP, r, hf, st->beta, st->a);
+      tc_fence_before();
+      group_issue<F, kJobUpdate>(a, sm, g, gt, dP, st);
       // after MMA3: next operand X_t = r(D_X)
       if (!(ok = wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status))) break;
       tc_fence_after();
       if (t + 1 < a.K) {
-        tmem_row_to_op<F, false, false>(tX, Xs, r, 1.f, 0.f);
-        signal_mma(sm.bar_epi(g));
+        tmem_row_to_op<F, false>(tX, tX, Xs, r, hf, 1.f);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr);
       }
     }
     if (!ok) break;
 
+    // X_s is free now (and S_s unless it stages O): start the next tile's loads
+    mg_issued = false;
+    if (gt == 0 && nxt->blk >= 0 && !a.has_o) {
+      issue_mg(a, sm, g, *nxt);
+      mg_issued = true;
+    }
+    __syncwarp();
+
     // ---- epilogue: O = D_X;  W <- W - lr O
+    if (has_w && !wait_or_abort(sm.bar_w(g), it & 1u, sm, a.status)) break;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       float v[32];
-      tmem_ld32(tX + 32 * i, v);
+      tmem_ld32(tX + 64 * hf + 32 * i, v);
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t off = chunk_off(r, 4 * i + j);
-        float o[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = v[8 * j + e];
-        if (a.has_o) *reinterpret_cast<uint4 *>(Xs + off) = pack8_bf16(o);
-        if (a.has_w) {
+        const uint32_t off = hf * kHalf + sw128_off(r, 4 * i + j);
+        const float *o = v + 8 * j;
+        if (a.has_o) *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(o);
+        if (has_w) {
           float w[8];
           unpack8(*reinterpret_cast<const uint4 *>(Ws + off), w);
 #pragma unroll
@@ -318,74 +473,17 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       }
     }
     fence_proxy_async_smem();
+    tc_fence_before();
     named_bar_sync(bar_id, kGroupThreads);
     if (gt == 0) {
-      if (a.has_o) store_tile(a.tmaps + b.tmap[kRoleOut], Xs, tc.x0, tc.y0, b.cols);
-      if (a.has_w) store_tile(a.tmaps + b.tmap[kRoleW], Ws, tc.x0, tc.y0, b.cols);
+      if (a.has_o) store_tile(a.tmaps + cur->tm[kRoleOut], Ss, cur->x0, cur->y0, cur->cols);
+      if (has_w) store_tile(a.tmaps + cur->tm[kRoleW], Ws, cur->x0, cur->y0, cur->cols);
       bulk_commit();
+      *cur = *nxt;
     }
+    __syncwarp();
   }
   if (gt == 0) bulk_wait0();
-}
-
-// ------------------------------------------------------------------ MMA issuer
-__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk) {
-  // K-major operand: 128 rows x 128 bf16, two swizzled 64-column halves;
-  // k-step kk covers columns 16kk..16kk+15.
-  return sw128_desc(base + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
-}
-__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk) {
-  // The same storage read MN-major (rows are K): k-step kk covers rows
-  // 16kk..16kk+15; the two 64-column halves are kHalf apart.
-  return sw128_desc(base + kk * 2048, kHalf, 1024);
-}
-
-template <int F>
-__device__ void mma_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem) {
-  const int64_t grid = gridDim.x;
-  int64_t jobs[2], done[2] = {0, 0};
-  for (int g = 0; g < 2; ++g) {
-    const int64_t first = blockIdx.x + g * grid;
-    const int64_t tiles = first < a.n_tiles ? (a.n_tiles - first + 2 * grid - 1) / (2 * grid) : 0;
-    jobs[g] = tiles * 3 * a.K;
-  }
-  const uint32_t idesc1 = idesc_f16(128, 128, F, 0, 0, 0);
-  const uint32_t idesc3 = idesc_f16(128, 128, F, 0, 1, 0);
-  uint32_t idle = 0;
-  while (done[0] < jobs[0] || done[1] < jobs[1]) {
-    bool progressed = false;
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      if (done[g] >= jobs[g] || !mbar_try_wait(sm.bar_epi(g), static_cast<uint32_t>(done[g] & 1))) continue;
-      tc_fence_after();
-      const int type = static_cast<int>(done[g] % 3);
-      const int t = static_cast<int>((done[g] / 3) % a.K);
-      const uint32_t xs = smem_u32(sm.x(g)), ss = smem_u32(sm.s(g));
-      const uint32_t dP = tmem + 256u * g, dX = dP + 128u;
-      if (type == 0) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(dP, desc_k(xs, kk), desc_k(xs, kk), idesc1, kk > 0);
-      } else if (type == 1) {
-        const ResidentStep &st = a.step[t];
-        const uint32_t idesc2 = idesc_f16(128, 128, F, 0, 0, st.neg2);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(dP, desc_k(ss, kk), desc_k(ss, kk), idesc2, st.acc2 | (kk > 0));
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(dX, desc_k(ss, kk), desc_mn(xs, kk), idesc3, 1u);
-      }
-      mma_commit(sm.bar_mma(g));
-      ++done[g];
-      progressed = true;
-    }
-    if (progressed) {
-      idle = 0;
-    } else if (++idle > kSpinLimit || ((idle & 1023u) == 1023u && *sm.abort_flag())) {
-      if (!*sm.abort_flag()) set_status(a.status, HIMUON_ERR_TIMEOUT);
-      *sm.abort_flag() = 1;
-      break;
-    }
-  }
 }
 
 template <int F>
@@ -397,30 +495,40 @@ __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_c
   if (threadIdx.x == 0) {
     for (int g = 0; g < 2; ++g) {
       mbar_init(sm.bar_ld(g), 1);
+      mbar_init(sm.bar_w(g), 1);
       mbar_init(sm.bar_mma(g), 1);
-      mbar_init(sm.bar_epi(g), kGroupThreads);
     }
     *sm.abort_flag() = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == 0) {
     tmem_alloc(sm.tmem_slot(), 512);
     tmem_relinquish();
+  }
+  if (use_smem_blocks(args)) {
+    for (int i = threadIdx.x; i < args.n_blocks; i += blockDim.x) {
+      const DevBlock &b = args.blocks[i];
+      SBlock &d = sm.blocks()[i];
+      d.tile_begin = static_cast<int32_t>(b.tile_begin);
+      d.cols = b.cols;
+      d.tiles_c = static_cast<uint16_t>(b.tiles_c);
+      d.T = static_cast<uint16_t>(b.T);
+#pragma unroll
+      for (int r = 0; r < kNumRoles; ++r) d.tm[r] = static_cast<int16_t>(b.tmap[r]);
+      d.pad = 0;
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
-  if (warp < kMmaWarp) {
-    group_main<F>(args, sm, tmem, warp >> 2);
-  } else if ((threadIdx.x & 31) == 0) {
-    mma_main<F>(args, sm, tmem);
-  }
+  group_main<F>(args, sm, tmem, warp / kGroupWarps);
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) {
+  if (warp == 0) {
     __syncwarp();
     tmem_dealloc(tmem, 512);
   }
@@ -429,11 +537,12 @@ __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_c
 }  // namespace
 
 int resident_smem_bytes() { return static_cast<int>(kSmemBytes); }
+int resident_max_smem_blocks() { return kMaxSmemBlocks; }
 
 void make_resident_steps(ResidentArgs &args, const float *coeffs, int K) {
   // MMA2 leaves D_P = B / beta with beta = b (beta = 1 when b = 0, in which
   // case MMA2 overwrites A with c A^2): S = r(sqrt|c / beta| A) and the sign of
-  // c / beta goes on MMA2's A operand.  MMA3 then adds r(beta D_P + (a-1) I) X.
+  // c / beta goes on MMA2's A operand.  MMA3 then forms r(beta D_P + a I) X.
   for (int t = 0; t < K; ++t) {
     const double a = coeffs[3 * t], b = coeffs[3 * t + 1], c = coeffs[3 * t + 2];
     const double beta = (b != 0.0) ? b : 1.0;
@@ -443,7 +552,7 @@ void make_resident_steps(ResidentArgs &args, const float *coeffs, int K) {
     st.neg2 = ratio < 0.0 ? 1u : 0u;
     st.acc2 = (b != 0.0) ? 1u : 0u;
     st.beta = static_cast<float>(beta);
-    st.am1 = static_cast<float>(a - 1.0);
+    st.a = static_cast<float>(a);
   }
 }
 

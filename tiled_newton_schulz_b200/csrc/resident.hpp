@@ -14,8 +14,8 @@ constexpr int kMaxSteps = 16;
 // make_resident_steps() for their meaning.
 struct ResidentStep {
   float s;          // S = r(s * A) feeds MMA2
-  float beta;       // Bop = r(beta * D_P + am1 * I) feeds MMA3
-  float am1;        // a_t - 1
+  float beta;       // Bop = r(beta * D_P + a * I) feeds MMA3
+  float a;          // a_t
   uint32_t neg2;    // MMA2 negates its A operand (c_t / beta < 0)
   uint32_t acc2;    // MMA2 accumulates onto A (b_t != 0)
 };
@@ -29,6 +29,7 @@ struct ResidentArgs {
   int32_t mode;     // 0: NS in -> out; 1: momentum step
   int32_t has_w, has_o;
   int32_t op_fmt;   // tensor-core operand type: 0 fp16, 1 bf16
+  int32_t smem_blocks;  // 1: the block table fits the kernel's compact shared-memory copy
   float mu, lr, eps, safety;
   ResidentStep step[kMaxSteps];
   int *status;
@@ -38,6 +39,7 @@ struct ResidentArgs {
 void make_resident_steps(ResidentArgs &args, const float *coeffs, int K);
 
 int resident_smem_bytes();
+int resident_max_smem_blocks();
 cudaError_t launch_ns_resident(const ResidentArgs &args, int grid, cudaStream_t stream);
 
 }  // namespace himuon
