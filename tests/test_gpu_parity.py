@@ -8,12 +8,16 @@ Tolerances (stated for the two arithmetic paths):
 * fp32 CUDA-core path: per-tile relative Frobenius error <= 1e-4.
 * bf16/fp16 tensor-core path: per-tile relative Frobenius error <= 3e-2, and
   sorted singular values of every checked tile within 0.05 of the oracle's.
-  Exception, bf16 operands only: a tile whose short side is below 64 (a thin
-  ragged edge strip) is held to 4e-2.  Rounding the operands to bf16 (8
-  significant bits) alone gives up to 3.0% on 44 x 128 strips in a CPU
-  emulation of the kernel's arithmetic (and 3.4% for Algorithm 1's own
-  all-bf16 loop), independent of any indexing; fp16 operands (11 bits) give
-  0.4% there and are held to 3e-2 everywhere.
+  Exception, bf16 operands only, for small tiles: short side 16..63 is held
+  to 4e-2 (singular values within 0.1) and short side below 16 to 8e-2
+  (singular values not checked).  Rounding the operands to bf16 (8 significant bits)
+  alone gives these errors in a CPU emulation of the kernel's arithmetic on
+  seeded Gaussian tiles (max over 20 draws): 3.0% on 44 x 128, 2.3% on
+  32 x 32, 4.0% on 32 x 6, 5.5% on 4 x 32, 6.6% on 2 x 3 -- independent of
+  any indexing; fp16 operands (11 bits) give 0.4%, 0.3%, 0.5%, 0.8%, 1.2% on
+  the same tiles and are held to 3e-2 everywhere.  The largest singular-value
+  deviation over the same draws is 0.047 on 32 x 32 bf16 tiles (a test that
+  samples 64 such tiles sees up to ~0.08) against 0.008 in fp16.
 * the stored momentum M' = mu M + G: within one bf16 ulp of the fp64 value.
 * tile placement: bit-exact (integer-coded tiles).
 """
@@ -30,7 +34,7 @@ pytestmark = pytest.mark.gpu
 QUINTIC = inputs.QUINTIC
 C32 = [tuple(float(np.float32(v)) for v in QUINTIC)] * 5   # the fp32 values the library receives
 TOL16, TOL32, SVTOL = 3e-2, 1e-4, 0.05
-TOL16_THIN_BF16 = 4e-2
+TOL16_THIN_BF16, TOL16_TINY_BF16 = 4e-2, 8e-2
 
 
 @pytest.fixture(scope="module")
@@ -49,10 +53,23 @@ def dev(x, dtype):
 def check16(Y, Yref, T, sv_sample=64, bf16=False):
     err = per_tile_errors(Y, Yref, T)
     H, W = Yref.shape
-    thin = np.array([min(h, w) < 64 for (_, _, h, w) in tiles(H, W, T)])
-    tol = np.where(thin & bf16, TOL16_THIN_BF16, TOL16)
+    short = np.array([min(h, w) for (_, _, h, w) in tiles(H, W, T)])
+    tol = np.full(err.shape, TOL16)
+    if bf16:
+        tol = np.where(short < 64, TOL16_THIN_BF16, tol)
+        tol = np.where(short < 16, TOL16_TINY_BF16, tol)
     assert np.all(err <= tol), f"max per-tile rel err {err.max():.4g}"
-    assert max_sv_diff(Y, Yref, T, sample=sv_sample) <= SVTOL
+    svtol = SVTOL
+    if bf16 and short.min() < 64:
+        svtol = 0.1
+    if bf16 and short.min() < 16:
+        keep = [t for t, sh in zip(tiles(H, W, T), short) if sh >= 16]
+        Yk = [(Y[r:r + h, c:c + w], Yref[r:r + h, c:c + w]) for (r, c, h, w) in keep]
+        worst = max((np.max(np.abs(np.linalg.svd(a, compute_uv=False) - np.linalg.svd(b, compute_uv=False)))
+                     for a, b in Yk), default=0.0)
+        assert worst <= svtol
+    else:
+        assert max_sv_diff(Y, Yref, T, sample=sv_sample) <= svtol
     return err.max()
 
 
@@ -72,6 +89,39 @@ def test_resident_tiled_ns(hm, H, W, compute):
     code = hm.BF16 if compute == "bf16" else hm.FP16
     xin, y = run_ns(hm, X, 128, code, torch.bfloat16)
     check16(y, oracle.ns_tiled(xin, 128, C32), 128, bf16=compute == "bf16")
+
+
+@pytest.mark.parametrize("compute", ["bf16", "fp16"])
+@pytest.mark.parametrize("T", [32, 64])
+@pytest.mark.parametrize("H,W", [(256, 384), (300, 500), (100, 70), (33, 65), (128, 4096)])
+def test_resident_packed_small_tiles(hm, H, W, T, compute):
+    """T = 64 / 32: two / four tiles share one 128 x 128 super-tile as diagonal blocks."""
+    X = inputs.gaussian((H, W), seed=7 * H + W + T)
+    code = hm.BF16 if compute == "bf16" else hm.FP16
+    xin, y = run_ns(hm, X, T, code, torch.bfloat16)
+    check16(y, oracle.ns_tiled(xin, T, C32), T, bf16=compute == "bf16")
+
+
+@pytest.mark.parametrize("T", [32, 64])
+def test_momentum_step_packed_small_tiles(hm, T):
+    rng = np.random.default_rng(T)
+    shapes = [(192, 320), (96, 128), (64, 33)]
+    w = [dev(0.02 * rng.standard_normal(sh), torch.bfloat16) for sh in shapes]
+    m = [dev(inputs.low_rank_plus_noise(*sh, inputs.sigma_inverse(8), 0.01, seed=300 + i), torch.bfloat16)
+         for i, sh in enumerate(shapes)]
+    g = [dev(inputs.low_rank_plus_noise(*sh, inputs.sigma_inverse(8), 0.01, seed=400 + i), torch.bfloat16)
+         for i, sh in enumerate(shapes)]
+    o = [torch.empty_like(x) for x in m]
+    w0, m0, g0 = [to_np(x) for x in w], [to_np(x) for x in m], [to_np(x) for x in g]
+    hm.momentum_step(w, m, g, 0.95, 0.02, hm.params(T, QUINTIC, steps=5, compute=hm.FP16), update_out=o)
+    assert hm.device_status() == 0
+    for i in range(len(shapes)):
+        W2, M2, O = oracle.momentum_step(w0[i], m0[i], g0[i], 0.95, 0.02, T, C32)
+        assert np.all(np.abs(to_np(m[i]) - M2) <= bf16_ulp(M2))
+        check16(to_np(o[i]), O, T)
+        wg = to_np(w[i])
+        bound = np.linalg.norm(0.5 * bf16_ulp(W2)) + float(np.float32(0.02)) * TOL16 * np.linalg.norm(O)
+        assert np.linalg.norm(wg - W2) <= bound
 
 
 def test_resident_zero_tile_and_scale(hm):
@@ -148,11 +198,12 @@ def test_momentum_step_resident(hm):
                 assert np.linalg.norm(wg[sl] - W2[sl]) <= bound
 
 
-def test_integer_coded_reassembly_bitexact(hm):
+@pytest.mark.parametrize("T", [32, 64, 128])
+def test_integer_coded_reassembly_bitexact(hm, T):
     """Tile t holds c_t P_t (signed permutation with its own shift and signs);
     the output keeps support and signs exactly, so any misplaced, swapped or
     transposed tile fails."""
-    H, W, T = 512, 384, 128
+    H, W = 512, 384
     X = np.zeros((H, W))
     for t, (r0, c0, h, w) in enumerate(oracle.tile_grid(H, W, T)):
         P = inputs.signed_permutation(T, shift=(7 * t) % T, sign_bits=(t * 2654435761) & 0x7FFFFFFF)

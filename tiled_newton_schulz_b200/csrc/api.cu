@@ -165,6 +165,7 @@ struct Plan {
   PathKind path = kPathStaged;
   std::vector<HostBlock> blocks;
   int64_t n_tiles = 0;
+  int pack = 1;                   // on-chip path: tiles per super-tile
   std::vector<TileClass> classes;
   void *dev = nullptr;            // [DevBlock...][CUtensorMap...][DevTile...]
   DevBlock *d_blocks = nullptr;
@@ -191,43 +192,55 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over a bf16 block: box 64 columns x 128 rows, 128-byte swizzle,
-// zero fill outside the block (the zero padding of ragged tiles).
-bool make_block_map(CUtensorMap *map, void *ptr, int64_t rows, int64_t cols, int64_t ld) {
+// 2-D map over a bf16 block for the on-chip kernel with `pack` tiles per
+// 128 x 128 super-tile: pack 1 -> box 64 columns x 128 rows, 128-byte swizzle;
+// pack 2 -> 64 x 64, 128-byte swizzle; pack 4 -> 32 x 32, 64-byte swizzle.
+// Zero fill outside the block (the zero padding of ragged tiles).
+bool make_block_map(CUtensorMap *map, void *ptr, int64_t rows, int64_t cols, int64_t ld, int pack) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
-  cuuint32_t box[2] = {64, 128};
+  const cuuint32_t T = static_cast<cuuint32_t>(128 / pack);
+  cuuint32_t box[2] = {pack == 1 ? 64u : T, pack == 1 ? 128u : T};
   cuuint32_t es[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUtensorMapSwizzle sw = pack == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 void *block_ptr(const himuon_mat &m, const HostBlock &b) {
   return static_cast<char *>(m.data) + (b.row0 * m.ld + b.col0) * static_cast<int64_t>(elem_size(m.dtype));
 }
 
-bool resident_ok(const CallMats &cm, const std::vector<HostBlock> &blocks, const himuon_ns_params &p) {
-  if (p.compute == HIMUON_FP32) return false;
+// Tiles per super-tile of the on-chip kernel for this call (1, 2 or 4), or 0
+// when the call needs the staged path: fp32 arithmetic, non-bf16 storage,
+// misaligned rows, or tiles that are neither 128 x 128 (edge tiles smaller),
+// 64 x 64, 32 x 32, nor a whole block of at most 128 x 128.
+int resident_pack(const CallMats &cm, const std::vector<HostBlock> &blocks, const himuon_ns_params &p) {
+  if (p.compute == HIMUON_FP32) return 0;
   for (int r = 0; r < kNumRoles; ++r) {
     if (!cm.role[r]) continue;
     for (int32_t i = 0; i < cm.n; ++i) {
       const himuon_mat &m = cm.role[r][i];
-      if (m.dtype != HIMUON_BF16) return false;
-      if ((m.ld * 2) % 16 != 0) return false;
+      if (m.dtype != HIMUON_BF16) return 0;
+      if ((m.ld * 2) % 16 != 0) return 0;
     }
   }
+  const int pack = (p.tile == 64 || p.tile == 32) ? 128 / p.tile : 1;
   for (const HostBlock &b : blocks) {
-    const bool single = b.T >= std::max(b.rows, b.cols) && std::max(b.rows, b.cols) <= 128;
-    if (!(b.T == 128 || single)) return false;
+    if (pack > 1) {
+      if (b.T != p.tile) return 0;
+    } else {
+      const bool single = b.T >= std::max(b.rows, b.cols) && std::max(b.rows, b.cols) <= 128;
+      if (!(b.T == 128 || single)) return 0;
+    }
     for (int r = 0; r < kNumRoles; ++r) {
       if (!cm.role[r]) continue;
-      if (reinterpret_cast<uintptr_t>(block_ptr(cm.role[r][b.mat], b)) % 16 != 0) return false;
+      if (reinterpret_cast<uintptr_t>(block_ptr(cm.role[r][b.mat], b)) % 16 != 0) return 0;
     }
   }
-  return true;
+  return pack;
 }
 
 std::string plan_key(int device, int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params &p) {
@@ -279,8 +292,10 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
   int rc = make_blocks(cm, splits, op == HIMUON_OP_NS_FULL || op == HIMUON_OP_GRAM_NS ? 0 : p.tile, plan->blocks,
                        &plan->n_tiles);
   if (rc) return rc;
-  const bool resident = op != HIMUON_OP_GRAM_NS && resident_ok(cm, plan->blocks, p);
+  const int pack = op != HIMUON_OP_GRAM_NS ? resident_pack(cm, plan->blocks, p) : 0;
+  const bool resident = pack > 0;
   plan->path = resident ? kPathResident : kPathStaged;
+  plan->pack = resident ? pack : 1;
 
   std::vector<DevBlock> dblocks(plan->blocks.size());
   std::vector<CUtensorMap> tmaps;
@@ -293,7 +308,7 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
     d.tiles_c = static_cast<int32_t>(b.tiles_c);
     d.rows = static_cast<int32_t>(b.rows);
     d.cols = static_cast<int32_t>(b.cols);
-    d.T = resident ? 128 : static_cast<int32_t>(b.T);
+    d.T = resident ? 128 / pack : static_cast<int32_t>(b.T);
     d.mat = b.mat;
     for (int r = 0; r < kNumRoles; ++r) {
       d.tmap[r] = -1;
@@ -304,7 +319,7 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
       d.dtype[r] = m.dtype;
       if (resident) {
         CUtensorMap tm;
-        if (!make_block_map(&tm, d.ptr[r], b.rows, b.cols, m.ld)) return HIMUON_ERR_CUDA;
+        if (!make_block_map(&tm, d.ptr[r], b.rows, b.cols, m.ld, pack)) return HIMUON_ERR_CUDA;
         d.tmap[r] = static_cast<int32_t>(tmaps.size());
         tmaps.push_back(tm);
       }
@@ -692,10 +707,16 @@ int run_resident(const Plan &plan, int op, const himuon_ns_params &p, float mu, 
   bool fits = static_cast<int>(plan.blocks.size()) <= resident_max_smem_blocks() && plan.n_tiles < (int64_t(1) << 31);
   for (const HostBlock &b : plan.blocks) fits = fits && b.tiles_c < 65536 && b.cols < (int64_t(1) << 31);
   a.smem_blocks = fits ? 1 : 0;
+  a.pack = plan.pack;
+  // HIMUON_TEST_STALL=1 exercises the device timeout path (tests only): the
+  // call then ends with HIMUON_ERR_TIMEOUT in the device status word.
+  const char *stall = getenv("HIMUON_TEST_STALL");
+  a.test_stall = (stall && stall[0] == '1') ? 1 : 0;
   make_resident_steps(a, p.coeffs, p.steps);
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, plan.device);
-  const int64_t want = (plan.n_tiles + 1) / 2;
+  const int64_t n_super = (plan.n_tiles + plan.pack - 1) / plan.pack;
+  const int64_t want = (n_super + 1) / 2;
   const int grid = static_cast<int>(std::min<int64_t>(sms, want));
   return launch_ns_resident(a, grid, stream) == cudaSuccess ? HIMUON_OK : HIMUON_ERR_CUDA;
 }
@@ -887,7 +908,7 @@ int64_t himuon_workspace_size(const himuon_mat *mats, int32_t n, const himuon_sp
   const int64_t tile = (op == HIMUON_OP_NS_FULL || op == HIMUON_OP_GRAM_NS) ? 0 : p->tile;
   rc = make_blocks(cm, splits, tile, blocks, &n_tiles);
   if (rc) return rc;
-  if (op != HIMUON_OP_GRAM_NS && resident_ok(cm, blocks, *p)) return 0;
+  if (op != HIMUON_OP_GRAM_NS && resident_pack(cm, blocks, *p) > 0) return 0;
   // staged: one tile of the largest class is the minimum; a full chunk of every
   // class makes the call run in one chunk per class.
   int64_t need = 0;

@@ -6,6 +6,11 @@
 // Tiles up to 128 x 128 are zero-padded to 128 x 128 (exactly the same map: a
 // zero border stays zero through X X^T, A^2 and B X and leaves ||X||_F alone;
 // and the transpose of a tall tile is not needed because NS(X^T) = NS(X)^T).
+// For T = 64 and T = 32, P = 128 / T consecutive tiles share one 128 x 128
+// "super-tile" as diagonal blocks, each normalised by its own norm: X X^T,
+// A^2 and B X of a block-diagonal matrix are block-diagonal with exactly the
+// blocks' own products (the off-diagonal zeros stay exact zeros in fp32), so
+// each block goes through exactly its own map.
 //
 // One persistent CTA per SM runs two independent tile "groups" of 8 warps
 // (two per TMEM lane quarter, each owning 64 of a row's 128 columns), so that
@@ -53,7 +58,9 @@ constexpr uint32_t kHalf = 16384;          // one 64-column, 128-row swizzled ha
 constexpr uint32_t kOffX = 0, kOffS = 32768, kOffW = 65536, kGroupBytes = 98304;
 constexpr uint32_t kOffBars = 2 * kGroupBytes;
 constexpr int kMaxSmemBlocks = 256;        // block tables up to this size live in shared memory
-constexpr uint32_t kOffBlocks = kOffBars + 512;
+constexpr int kMaxPack = 4;                // tiles per super-tile (T = 32)
+constexpr uint32_t kOffCoords = kOffBars + 512;                    // 2 groups x 2 x kMaxPack TileCoords
+constexpr uint32_t kOffBlocks = kOffCoords + 2 * 2 * kMaxPack * 32;
 constexpr uint32_t kSmemBytes = kOffBlocks + kMaxSmemBlocks * 24 + 1024;   // + alignment slack
 
 struct TileCoord {
@@ -72,6 +79,7 @@ struct SBlock {
   int32_t pad;
 };
 static_assert(sizeof(SBlock) == 24, "SBlock layout");
+static_assert(sizeof(TileCoord) == 32, "TileCoord layout");
 
 struct Smem {
   uint8_t *base;
@@ -82,20 +90,29 @@ struct Smem {
   __device__ uint64_t *bar_ld(int g) const { return bar(g, 0); }    // M (or input) and G landed
   __device__ uint64_t *bar_w(int g) const { return bar(g, 1); }     // W landed
   __device__ uint64_t *bar_mma(int g) const { return bar(g, 2); }   // the group's MMA job finished
+  __device__ uint64_t *bar_never(int g) const { return bar(g, 3); } // never arrived on (stall self-test)
   __device__ float *red(int g) const { return reinterpret_cast<float *>(base + kOffBars + 64) + kGroupWarps * g; }
   __device__ uint32_t *tmem_slot() const { return reinterpret_cast<uint32_t *>(base + kOffBars + 128); }
   __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(base + kOffBars + 132); }
   __device__ SBlock *blocks() const { return reinterpret_cast<SBlock *>(base + kOffBlocks); }
-  // current / next tile coordinates of group g (read and written by its issuing thread only)
+  // current (i = 0) / next (i = 1) super-tile's tile coordinates of group g,
+  // kMaxPack each (read and written by the group's issuing thread only)
   __device__ TileCoord *coord(int g, int i) const {
-    return reinterpret_cast<TileCoord *>(base + kOffBars + 256) + 2 * g + i;
+    return reinterpret_cast<TileCoord *>(base + kOffCoords) + (2 * g + i) * kMaxPack;
   }
 };
 
+// Bounded wait that also gives up as soon as another thread of the CTA has
+// raised the abort flag (after its own wait timed out).
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, const Smem &sm, int *status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023u) == 1023u && *sm.abort_flag()) return false;
+    if ((i & 255u) == 0) {
+      if (*sm.abort_flag()) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
   }
   set_status(status, HIMUON_ERR_TIMEOUT);
   *sm.abort_flag() = 1;
@@ -197,7 +214,7 @@ __device__ __forceinline__ bool use_smem_blocks(const ResidentArgs &a) {
 
 // Block of `tile` by binary search over tile_begin, in the shared-memory copy
 // of the block table when it fits there (a few shared loads), else in global.
-__device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, const Smem &sm, int64_t tile) {
+__device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, const Smem &sm, int64_t tile, int hint = -1) {
   TileCoord t;
   t.blk = -1;
   t.x0 = t.y0 = t.cols = 0;
@@ -207,6 +224,11 @@ __device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, const Sm
   int lo = 0, hi = a.n_blocks - 1;
   if (use_smem_blocks(a)) {
     const SBlock *sb = sm.blocks();
+    if (hint >= 0) {  // the tile right after one in block `hint`: same block or a later one
+      lo = hint;
+      while (lo < hi && sb[lo + 1].tile_begin <= tile) ++lo;
+      hi = lo;
+    }
     while (lo < hi) {  // last block with tile_begin <= tile
       const int mid = (lo + hi + 1) >> 1;
       if (sb[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
@@ -236,30 +258,78 @@ __device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, const Sm
   return t;
 }
 
-__device__ __forceinline__ void load_tile(const CUtensorMap *m, uint8_t *dst, int32_t x0, int32_t y0, uint64_t *bar) {
-  tma_load_2d(dst, m, x0, y0, bar);
-  tma_load_2d(dst + kHalf, m, x0 + 64, y0, bar);
+// Staged tiles in shared memory (TMA boxes; the swizzle is applied by TMA):
+//   P = 1: one 128 x 128 tile as two 64-column halves, 128-byte swizzle;
+//   P = 2: sub-tile j (64 x 64) at j * 8 KB, 128-byte rows, 128-byte swizzle;
+//   P = 4: sub-tile j (32 x 32) at j * 2 KB, 64-byte rows, 64-byte swizzle.
+template <int P>
+__device__ __forceinline__ uint32_t stage_off(uint32_t j, uint32_t row, uint32_t c) {
+  if (P == 1) return (c >> 3) * kHalf + sw128_off(row, c & 7u);
+  if (P == 2) return j * 8192u + sw128_off(row, c);
+  return j * 2048u + row * 64u + ((c ^ ((row >> 1) & 3u)) << 4);
 }
-__device__ __forceinline__ void store_tile(const CUtensorMap *m, const uint8_t *src, int32_t x0, int32_t y0,
-                                           int32_t cols) {
-  tma_store_2d(m, src, x0, y0);
-  if (x0 + 64 < cols) tma_store_2d(m, src + kHalf, x0 + 64, y0);
+template <int P>
+__device__ __forceinline__ void load_tile(const CUtensorMap *m, uint8_t *dst, const TileCoord &t, int j,
+                                          uint64_t *bar) {
+  if (P == 1) {
+    tma_load_2d(dst, m, t.x0, t.y0, bar);
+    tma_load_2d(dst + kHalf, m, t.x0 + 64, t.y0, bar);
+  } else {
+    tma_load_2d(dst + stage_off<P>(j, 0, 0), m, t.x0, t.y0, bar);
+  }
 }
-__device__ __forceinline__ void prefetch_tile(const CUtensorMap *m, int32_t x0, int32_t y0, int32_t cols) {
-  tma_prefetch_l2_2d(m, x0, y0);
-  if (x0 + 64 < cols) tma_prefetch_l2_2d(m, x0 + 64, y0);
+template <int P>
+__device__ __forceinline__ void store_tile(const CUtensorMap *m, const uint8_t *src, const TileCoord &t, int j) {
+  if (P == 1) {
+    tma_store_2d(m, src, t.x0, t.y0);
+    if (t.x0 + 64 < t.cols) tma_store_2d(m, src + kHalf, t.x0 + 64, t.y0);
+  } else {
+    tma_store_2d(m, src + stage_off<P>(j, 0, 0), t.x0, t.y0);
+  }
+}
+template <int P>
+__device__ __forceinline__ void prefetch_tile(const CUtensorMap *m, const TileCoord &t) {
+  tma_prefetch_l2_2d(m, t.x0, t.y0);
+  if (P == 1 && t.x0 + 64 < t.cols) tma_prefetch_l2_2d(m, t.x0 + 64, t.y0);
 }
 
-// M (or the NS input) -> X_s and, for a momentum step, G -> S_s.
-__device__ __forceinline__ void issue_mg(const ResidentArgs &a, const Smem &sm, int g, const TileCoord &t) {
+// bytes one role's TMA boxes bring in for tile coordinate t
+template <int P>
+__device__ __forceinline__ uint32_t tile_bytes() { return P == 1 ? 2 * kHalf : (128 / P) * (128 / P) * 2; }
+
+// M (or the NS input) -> X_s and, for a momentum step, G -> S_s, for every
+// tile of the super-tile.
+template <int P>
+__device__ __forceinline__ void issue_mg(const ResidentArgs &a, const Smem &sm, int g, const TileCoord *t) {
   const bool step_mode = a.mode == 1;
-  mbar_arrive_expect_tx(sm.bar_ld(g), step_mode ? 4 * kHalf : 2 * kHalf);
-  load_tile(a.tmaps + t.tm[kRoleIn], sm.x(g), t.x0, t.y0, sm.bar_ld(g));
-  if (step_mode) load_tile(a.tmaps + t.tm[kRoleG], sm.s(g), t.x0, t.y0, sm.bar_ld(g));
+  uint32_t bytes = 0;
+#pragma unroll
+  for (int j = 0; j < P; ++j)
+    if (t[j].blk >= 0) bytes += (step_mode ? 2 : 1) * tile_bytes<P>();
+  mbar_arrive_expect_tx(sm.bar_ld(g), bytes);
+#pragma unroll
+  for (int j = 0; j < P; ++j) {
+    if (t[j].blk < 0) continue;
+    load_tile<P>(a.tmaps + t[j].tm[kRoleIn], sm.x(g), t[j], j, sm.bar_ld(g));
+    if (step_mode) load_tile<P>(a.tmaps + t[j].tm[kRoleG], sm.s(g), t[j], j, sm.bar_ld(g));
+  }
 }
-__device__ __forceinline__ void issue_w(const ResidentArgs &a, const Smem &sm, int g, const TileCoord &t) {
-  mbar_arrive_expect_tx(sm.bar_w(g), 2 * kHalf);
-  load_tile(a.tmaps + t.tm[kRoleW], sm.w(g), t.x0, t.y0, sm.bar_w(g));
+template <int P>
+__device__ __forceinline__ void issue_w(const ResidentArgs &a, const Smem &sm, int g, const TileCoord *t) {
+  uint32_t bytes = 0;
+#pragma unroll
+  for (int j = 0; j < P; ++j)
+    if (t[j].blk >= 0) bytes += tile_bytes<P>();
+  mbar_arrive_expect_tx(sm.bar_w(g), bytes);
+#pragma unroll
+  for (int j = 0; j < P; ++j)
+    if (t[j].blk >= 0) load_tile<P>(a.tmaps + t[j].tm[kRoleW], sm.w(g), t[j], j, sm.bar_w(g));
+}
+// coordinates of the P tiles of super-tile `st` (tile P st + j; blk = -1 past the end)
+template <int P>
+__device__ __forceinline__ void decode_super(const ResidentArgs &a, const Smem &sm, int64_t st, TileCoord *out) {
+#pragma unroll
+  for (int j = 0; j < P; ++j) out[j] = decode_tile(a, sm, P * st + j, j == 0 ? -1 : out[j - 1].blk);
 }
 
 // ------------------------------------------------------------------ MMA issue
@@ -284,16 +354,20 @@ enum Job { kJobGram = 0, kJobSquare = 1, kJobUpdate = 2 };
 template <int F, int JOB>
 __device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st);
 
+// The barrier also ORs the threads' failure flags: if any thread of the group
+// saw a wait give up, nothing is issued and every thread learns to stop
+// (returns true), at the same point.
 template <int F, int JOB>
-__device__ __forceinline__ void group_issue(const ResidentArgs &a, const Smem &sm, int g, int gt, uint32_t dP,
-                                            const ResidentStep *st) {
-  named_bar_sync(1 + g, kGroupThreads);
-  if (gt >= 32) return;
+__device__ __forceinline__ bool group_issue(const ResidentArgs &a, const Smem &sm, int g, int gt, uint32_t dP,
+                                            const ResidentStep *st, bool bad) {
+  if (named_bar_or(1 + g, kGroupThreads, bad)) return true;
+  if (gt >= 32) return false;
   // Lanes 1..31 of the issuing warp wait here for lane 0: if they went on to
   // spin on the completion barrier, the warp would interleave their
   // (suspending) try_wait with lane 0's issue and delay the MMAs.
   if (gt == 0) group_issue_mmas<F, JOB>(sm, g, dP, st);
   __syncwarp();
+  return false;
 }
 
 template <int F, int JOB>
@@ -324,14 +398,18 @@ __device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t
 }
 
 // ------------------------------------------------------------------ one tile group
-template <int F>
+// P tiles of edge T = 128 / P per super-tile (P = 1: one 128-tile).
+template <int F, int P>
 __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem, int g) {
+  constexpr uint32_t T = 128 / P;
   const int gt = threadIdx.x - g * kGroupThreads;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wig = warp - g * kGroupWarps;              // warp in group, 0..7
   const uint32_t q = static_cast<uint32_t>(warp & 3);  // TMEM lane quarter
   const uint32_t hf = static_cast<uint32_t>(wig >> 2); // column half owned by this thread
-  const uint32_t r = q * 32 + lane;                    // tile row
+  const uint32_t r = q * 32 + lane;                    // super-tile row
+  const uint32_t jr = P == 1 ? 0u : r / T;             // this row's tile (diagonal block)
+  const uint32_t rr = r - jr * T;                      // ... and its row inside that tile
   const uint32_t dP = tmem + 256u * g;                 // D_P (lane 0); D_X = dP + 128
   const uint32_t tP = dP + ((q * 32) << 16);           // this warp's lanes of D_P
   const uint32_t tX = tP + 128u;                       // ... and of D_X
@@ -340,41 +418,66 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
   const bool step_mode = a.mode == 1;
   const bool has_w = step_mode && a.has_w;
   const int64_t grid = gridDim.x;
+  const int64_t n_super = (a.n_tiles + P - 1) / P;
   uint32_t it = 0, job = 0;
-  bool mg_issued = false;   // (issuing thread) this tile's M/G loads went out during the previous tile
+  bool mg_issued = false;   // (issuing thread) this super-tile's M/G loads went out during the previous one
+  // (issuing thread) phases armed on / waited for on bar_ld, bar_w and bar_mma,
+  // so that an aborted tile can wait for its own copies and MMAs in flight
+  uint32_t ld_armed = 0, ld_seen = 0, w_armed = 0, w_seen = 0, mma_armed = 0, mma_seen = 0;
+  // Self-test of the timeout path: one group waits on a barrier that nothing
+  // arrives on, times out, records HIMUON_ERR_TIMEOUT and makes the CTA abort.
+  if (a.test_stall && blockIdx.x == 0 && g == 0) wait_or_abort(sm.bar_never(g), 0, sm, a.status);
+  const bool stalled = *sm.abort_flag() != 0;
   TileCoord *cur = sm.coord(g, 0), *nxt = sm.coord(g, 1);
-  if (gt == 0) *cur = decode_tile(a, sm, blockIdx.x + g * grid);
+  if (gt == 0) decode_super<P>(a, sm, blockIdx.x + g * grid, cur);
 
-  for (int64_t tile = blockIdx.x + g * grid; tile < a.n_tiles; tile += 2 * grid, ++it) {
+  for (int64_t st = blockIdx.x + g * grid; st < n_super && !stalled; st += 2 * grid, ++it) {
+    // this row's tile exists (the last super-tile may hold fewer than P tiles)
+    const bool row_valid = P == 1 || P * st + jr < a.n_tiles;
     if (gt == 0) {
-      bulk_wait_read0();  // the previous tile's stores have finished reading S_s / W_s
-      if (!mg_issued) issue_mg(a, sm, g, *cur);
-      if (has_w) issue_w(a, sm, g, *cur);
+      bulk_wait_read0();  // the previous super-tile's stores have finished reading S_s / W_s
+      if (!mg_issued) {
+        issue_mg<P>(a, sm, g, cur);
+        ++ld_armed;
+      }
+      if (has_w) {
+        issue_w<P>(a, sm, g, cur);
+        ++w_armed;
+      }
     }
     __syncwarp();
-    if (!wait_or_abort(sm.bar_ld(g), it & 1u, sm, a.status)) break;
+    // A failed wait is only recorded here; the group stops together at its
+    // next barrier (a thread leaving alone would strand the others there).
+    bool bad = !wait_or_abort(sm.bar_ld(g), it & 1u, sm, a.status);
+    if (!bad) ++ld_seen;
 
     // ---- prologue: M' = mu M + G (or the plain input), ||.||_F, fp32 copy to D_X.
     // M' (bf16, for the write-back) replaces G in S_s, so X_s is free for X_0 at once.
+    // Columns outside this row's diagonal block are zero.
     float sumsq = 0.f;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       float v[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t off = hf * kHalf + sw128_off(r, 4 * i + j);
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t cg = 8 * hf + 4 * i + k;         // 8-column chunk of the super-tile row
         float m[8];
-        unpack8(*reinterpret_cast<const uint4 *>(Xs + off), m);
-        if (step_mode) {
-          float gg[8];
-          unpack8(*reinterpret_cast<const uint4 *>(Ss + off), gg);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) m[e] = fmaf(a.mu, m[e], gg[e]);
-          *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(m);
+        for (int e = 0; e < 8; ++e) m[e] = 0.f;
+        if (P == 1 || ((8 * cg) / T == jr && row_valid)) {
+          const uint32_t off = stage_off<P>(jr, rr, cg - jr * (T / 8));
+          unpack8(*reinterpret_cast<const uint4 *>(Xs + off), m);
+          if (step_mode) {
+            float gg[8];
+            unpack8(*reinterpret_cast<const uint4 *>(Ss + off), gg);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m[e] = fmaf(a.mu, m[e], gg[e]);
+            *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(m);
+          }
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          v[8 * j + e] = m[e];
+          v[8 * k + e] = m[e];
           sumsq = fmaf(m[e], m[e], sumsq);
         }
       }
@@ -384,15 +487,19 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     sumsq = warp_sum(sumsq);
     if (lane == 0) sm.red(g)[wig] = sumsq;
     if (step_mode) fence_proxy_async_smem();
-    named_bar_sync(bar_id, kGroupThreads);   // M' complete in S_s, partial sums visible, M read
+    // M' complete in S_s, partial sums visible, M read
+    if (named_bar_or(bar_id, kGroupThreads, bad)) break;
     if (step_mode && gt == 0) {
-      store_tile(a.tmaps + cur->tm[kRoleIn], Ss, cur->x0, cur->y0, cur->cols);
+#pragma unroll
+      for (int j = 0; j < P; ++j)
+        if (cur[j].blk >= 0) store_tile<P>(a.tmaps + cur[j].tm[kRoleIn], Ss, cur[j], j);
       bulk_commit();
     }
     __syncwarp();
-    float total = 0.f;
+    float total = 0.f;   // ||tile||^2 of this row's tile: the warps whose rows lie in it
 #pragma unroll
-    for (int i = 0; i < kGroupWarps; ++i) total += sm.red(g)[i];
+    for (int w = 0; w < kGroupWarps; ++w)
+      if (P == 1 || (32u * (w & 3)) / T == jr) total += sm.red(g)[w];
     const float rho = (sqrtf(total) + a.eps) * a.safety;
 
     // ---- X_0 = r(M' / rho) to X_s and (packed) to D_X
@@ -403,90 +510,121 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     __syncwarp();
     fence_proxy_async_smem();
     tc_fence_before();
-    group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr);
+    if (group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr, bad)) break;
+    ++mma_armed;
 
-    if (gt == 0) {   // next tile of this group, while MMA1 runs
-      *nxt = decode_tile(a, sm, tile + 2 * grid);
-      if (nxt->blk >= 0) {
-        prefetch_tile(a.tmaps + nxt->tm[kRoleIn], nxt->x0, nxt->y0, nxt->cols);
-        if (step_mode) prefetch_tile(a.tmaps + nxt->tm[kRoleG], nxt->x0, nxt->y0, nxt->cols);
-        if (has_w) prefetch_tile(a.tmaps + nxt->tm[kRoleW], nxt->x0, nxt->y0, nxt->cols);
+    if (gt == 0) {   // next super-tile of this group, while MMA1 runs
+      decode_super<P>(a, sm, st + 2 * grid, nxt);
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        if (nxt[j].blk < 0) continue;
+        prefetch_tile<P>(a.tmaps + nxt[j].tm[kRoleIn], nxt[j]);
+        if (step_mode) prefetch_tile<P>(a.tmaps + nxt[j].tm[kRoleG], nxt[j]);
+        if (has_w) prefetch_tile<P>(a.tmaps + nxt[j].tm[kRoleW], nxt[j]);
       }
     }
     __syncwarp();
 
-    bool ok = true;
-    for (int t = 0; t < a.K && ok; ++t) {
-      const ResidentStep *st = &a.step[t];
+    bool stop = false;
+    for (int t = 0; t < a.K && !stop; ++t) {
+      const ResidentStep *stp = &a.step[t];
       // after MMA1: S = r(s A) to S_s and (packed) to D_X
-      if (!(ok = wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status))) break;
+      bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
+      if (!bad) ++mma_seen;
       tc_fence_after();
-      tmem_row_to_op<F, true>(tP, tX, Ss, r, hf, st->s);
+      tmem_row_to_op<F, true>(tP, tX, Ss, r, hf, stp->s);
       fence_proxy_async_smem();
       tc_fence_before();
-      group_issue<F, kJobSquare>(a, sm, g, gt, dP, st);
+      if ((stop = group_issue<F, kJobSquare>(a, sm, g, gt, dP, stp, bad))) break;
+      ++mma_armed;
       // after MMA2: Bop = r(beta D_P + a I), packed in D_P
-      if (!(ok = wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status))) break;
+      bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
+      if (!bad) ++mma_seen;
       tc_fence_after();
-      tmem_row_to_tmem_op<F>(tP, r, hf, st->beta, st->a);
+      tmem_row_to_tmem_op<F>(tP, r, hf, stp->beta, stp->a);
       tc_fence_before();
-      group_issue<F, kJobUpdate>(a, sm, g, gt, dP, st);
+      if ((stop = group_issue<F, kJobUpdate>(a, sm, g, gt, dP, stp, bad))) break;
+      ++mma_armed;
       // after MMA3: next operand X_t = r(D_X)
-      if (!(ok = wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status))) break;
+      bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
+      if (!bad) ++mma_seen;
       tc_fence_after();
       if (t + 1 < a.K) {
         tmem_row_to_op<F, false>(tX, tX, Xs, r, hf, 1.f);
         fence_proxy_async_smem();
         tc_fence_before();
-        group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr);
+        if ((stop = group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr, bad))) break;
+        ++mma_armed;
       }
     }
-    if (!ok) break;
+    if (stop) break;
 
-    // X_s is free now (and S_s unless it stages O): start the next tile's loads
+    // X_s is free now (and S_s unless it stages O): start the next super-tile's loads
     mg_issued = false;
-    if (gt == 0 && nxt->blk >= 0 && !a.has_o) {
-      issue_mg(a, sm, g, *nxt);
+    if (gt == 0 && nxt[0].blk >= 0 && !a.has_o && !bad) {
+      issue_mg<P>(a, sm, g, nxt);
+      ++ld_armed;
       mg_issued = true;
     }
     __syncwarp();
 
-    // ---- epilogue: O = D_X;  W <- W - lr O
-    if (has_w && !wait_or_abort(sm.bar_w(g), it & 1u, sm, a.status)) break;
+    // ---- epilogue: O = D_X;  W <- W - lr O  (this row's diagonal block only)
+    if (has_w) {
+      const bool wbad = !wait_or_abort(sm.bar_w(g), it & 1u, sm, a.status);
+      if (!wbad) ++w_seen;
+      bad = bad || wbad;
+    }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      float v[32];
-      tmem_ld32(tX + 64 * hf + 32 * i, v);
-      tmem_wait_ld();
+      const uint32_t c32 = 2 * hf + i;                  // 32-column group of the super-tile row
+      if (P == 1 || ((32 * c32) / T == jr && row_valid)) {
+        float v[32];
+        tmem_ld32(tX + 32 * c32, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t off = hf * kHalf + sw128_off(r, 4 * i + j);
-        const float *o = v + 8 * j;
-        if (a.has_o) *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(o);
-        if (has_w) {
-          float w[8];
-          unpack8(*reinterpret_cast<const uint4 *>(Ws + off), w);
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t cg = 4 * c32 + k;
+          const uint32_t off = stage_off<P>(jr, rr, cg - jr * (T / 8));
+          const float *o = v + 8 * k;
+          if (a.has_o) *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(o);
+          if (has_w) {
+            float w[8];
+            unpack8(*reinterpret_cast<const uint4 *>(Ws + off), w);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) w[e] = fmaf(-a.lr, o[e], w[e]);
-          *reinterpret_cast<uint4 *>(Ws + off) = pack8_bf16(w);
+            for (int e = 0; e < 8; ++e) w[e] = fmaf(-a.lr, o[e], w[e]);
+            *reinterpret_cast<uint4 *>(Ws + off) = pack8_bf16(w);
+          }
         }
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    named_bar_sync(bar_id, kGroupThreads);
+    if (named_bar_or(bar_id, kGroupThreads, bad)) break;
     if (gt == 0) {
-      if (a.has_o) store_tile(a.tmaps + cur->tm[kRoleOut], Ss, cur->x0, cur->y0, cur->cols);
-      if (has_w) store_tile(a.tmaps + cur->tm[kRoleW], Ws, cur->x0, cur->y0, cur->cols);
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        if (cur[j].blk < 0) continue;
+        if (a.has_o) store_tile<P>(a.tmaps + cur[j].tm[kRoleOut], Ss, cur[j], j);
+        if (has_w) store_tile<P>(a.tmaps + cur[j].tm[kRoleW], Ws, cur[j], j);
+      }
       bulk_commit();
-      *cur = *nxt;
+#pragma unroll
+      for (int j = 0; j < P; ++j) cur[j] = nxt[j];
     }
     __syncwarp();
   }
-  if (gt == 0) bulk_wait0();
+  if (gt == 0) {
+    // After an abort: wait (bounded) for this group's own loads and MMAs still
+    // in flight, so that no copy lands in, and no MMA touches, memory the CTA
+    // is about to release.  Nothing is outstanding after a normal finish.
+    for (; ld_seen < ld_armed; ++ld_seen) mbar_wait(sm.bar_ld(g), ld_seen & 1u, a.status);
+    for (; w_seen < w_armed; ++w_seen) mbar_wait(sm.bar_w(g), w_seen & 1u, a.status);
+    for (; mma_seen < mma_armed; ++mma_seen) mbar_wait(sm.bar_mma(g), mma_seen & 1u, a.status);
+    bulk_wait0();
+  }
 }
 
-template <int F>
+template <int F, int P>
 __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_constant__ ResidentArgs args) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
@@ -497,6 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_c
       mbar_init(sm.bar_ld(g), 1);
       mbar_init(sm.bar_w(g), 1);
       mbar_init(sm.bar_mma(g), 1);
+      mbar_init(sm.bar_never(g), 1);
     }
     *sm.abort_flag() = 0;
     fence_mbar_init();
@@ -523,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
-  group_main<F>(args, sm, tmem, warp / kGroupWarps);
+  group_main<F, P>(args, sm, tmem, warp / kGroupWarps);
 
   tc_fence_before();
   __syncthreads();
@@ -556,19 +695,24 @@ void make_resident_steps(ResidentArgs &args, const float *coeffs, int K) {
   }
 }
 
-template <int F>
+template <int F, int P>
 static cudaError_t launch_fmt(const ResidentArgs &args, int grid, cudaStream_t stream) {
   // The shared-memory opt-in is per device; setting it again is cheap.
-  cudaError_t e = cudaFuncSetAttribute(ns_resident_kernel<F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(ns_resident_kernel<F, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   count_launch();
-  ns_resident_kernel<F><<<grid, kThreads, kSmemBytes, stream>>>(args);
+  ns_resident_kernel<F, P><<<grid, kThreads, kSmemBytes, stream>>>(args);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ns_resident(const ResidentArgs &args, int grid, cudaStream_t stream) {
-  return args.op_fmt == 0 ? launch_fmt<0>(args, grid, stream) : launch_fmt<1>(args, grid, stream);
+  const bool f16 = args.op_fmt == 0;
+  switch (args.pack) {
+    case 2: return f16 ? launch_fmt<0, 2>(args, grid, stream) : launch_fmt<1, 2>(args, grid, stream);
+    case 4: return f16 ? launch_fmt<0, 4>(args, grid, stream) : launch_fmt<1, 4>(args, grid, stream);
+    default: return f16 ? launch_fmt<0, 1>(args, grid, stream) : launch_fmt<1, 1>(args, grid, stream);
+  }
 }
 
 }  // namespace himuon

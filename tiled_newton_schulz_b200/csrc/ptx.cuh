@@ -1,8 +1,10 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA, tcgen05.
 //
-// Every wait on an mbarrier is bounded: after kSpinLimit polls it records
-// HIMUON_ERR_TIMEOUT in the device status word and returns false, so a lost
-// arrival can never hang the GPU.  Callers then skip the rest of their work.
+// Every wait on an mbarrier is bounded in time: after kWaitLimitNs of global
+// time it records HIMUON_ERR_TIMEOUT in the device status word and returns
+// false, so a lost arrival can never hang the GPU.  Callers then skip the rest
+// of their work (after waiting, again bounded, for their own copies and MMAs
+// in flight).
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -12,10 +14,15 @@
 
 namespace himuon {
 
-// ~ 2^22 polls of try_wait (each of which itself suspends for a while) is
-// far above any legitimate wait in these kernels (microseconds), and well
-// below a watchdog-scale stall.
-constexpr uint32_t kSpinLimit = 1u << 22;
+// Two seconds: far above any legitimate wait in these kernels (microseconds),
+// far below a watchdog-scale stall.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -63,8 +70,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t phase) {
 }
 // Bounded wait for the phase with parity `phase` to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, int *status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, phase)) return true;
+    if ((i & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) break;
+  }
   set_status(status, HIMUON_ERR_TIMEOUT_DEV);
   return false;
 }
@@ -75,6 +86,20 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also ORs a predicate over the participating threads:
+// every thread gets the same answer, so a group can agree to stop.
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(out)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return out != 0;
 }
 
 // ---------------------------------------------------------------- TMA
