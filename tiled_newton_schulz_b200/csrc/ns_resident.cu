@@ -21,14 +21,23 @@
 //   shared memory  X_s (16-bit iterate operand, 32 KB), S_s (16-bit operand, 32 KB), W_s (32 KB)
 //   tensor memory  D_P (128 cols fp32: A, then B / b), D_X (128 cols fp32: the iterate)
 // Per step the group runs three 128x128x128 MMAs, every A operand read from
-// TMEM and every B operand from shared memory:
-//   MMA1  D_P  = X X^T                          A: X (packed in D_X),   B: X_s (K-major)
-//   MMA2  D_P += sign(c/b) S S^T                A: S (packed in D_X),   B: S_s,  S = r(sqrt|c/b| A)
-//                                               -> D_P = A + (c/b) A^2 = B / b
-//   MMA3  D_X  = Bop X,  Bop = r(b D_P + a I)   A: Bop (packed in D_P), B: X_s (MN-major)
-// r() rounds to the 16-bit operand type (fp16 or bf16, chosen per call).
-// MMA3 forms the whole update X <- a X + B X = (a I + B) X with fp32
-// accumulation.  A 16-bit operand is packed two per 32-bit TMEM column in
+// TMEM and every B operand from shared memory.  The operand carries the
+// iterate scaled, Xg = g X with g = sqrt|c/b|, which is what lets S go to
+// the tensor cores without a multiply of its own:
+//   MMA1  D_P  = Xg Xg^T = g^2 A                 A: Xg (packed in D_X),  B: X_s (K-major)
+//   MMA2  D_P += sign(c/b) S S^T,  S = r(D_P)   A: S (packed in D_X),   B: S_s
+//                                               -> D_P = g^2 (A + (c/b) A^2) = g^2 B / b
+//   MMA3  D_X  = Bop Xg,  Bop = r((b/g^2) D_P + a I) = r(a I + B)
+//                                               A: Bop (packed in D_P), B: X_s (MN-major)
+// so D_X = g X_{t+1}, which is the next step's operand as it stands (a ratio
+// g_{t+1}/g_t is applied when the coefficients change; O = D_X / g).  r()
+// rounds to the 16-bit operand type (fp16 or bf16, chosen per call); every
+// operand is still one rounding of an fp32 value, with the relative error
+// bound of the unscaled iteration (g = 0.65 for the quintic coefficients keeps
+// fp16 operands far from its range limits).  MMA3 forms the whole update
+// X <- a X + B X = (a I + B) X with fp32 accumulation.  The conversions are
+// partly bound by the SM's arithmetic pipes, which is why S and X carry no
+// multiply and the diagonal a I is added only in the 32 columns that hold it.  A 16-bit operand is packed two per 32-bit TMEM column in
 // place: each thread, having read its 64 fp32 columns of a region, writes
 // their 16-bit values to the first 32 of those columns (nobody else reads
 // them), or into D_X while D_X holds nothing live.  Keeping A operands out of
@@ -42,6 +51,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
+
+#include <vector>
 
 #include "layout.hpp"
 #include "ptx.cuh"
@@ -185,23 +196,31 @@ __device__ __forceinline__ void tmem_row_to_op(uint32_t src, uint32_t pk, uint8_
 // Bop = r(beta * D_P + diag * I) for this thread's 64 columns of row r,
 // packed two per 32-bit word into TMEM columns [64 hf, 64 hf + 32) of D_P
 // (columns this thread has already read; nobody else reads them).
+// Row r = 32 q + lane: its diagonal element lies in column half r / 64 = q / 2,
+// 32-column chunk q % 2 of that half, position lane -- so whether a warp's
+// chunk holds it is uniform across the warp, and only that chunk pays for
+// the per-element test.
 template <int F>
 __device__ __forceinline__ void tmem_row_to_tmem_op(uint32_t taddr, uint32_t r, uint32_t hf, float beta, float diag) {
   const uint32_t c0 = 64u * hf;
-  const bool mine = (r >> 6) == hf;            // the diagonal element sits in this thread's columns
-  const uint32_t dl = (r & 63u);               // its position among them
+  const uint32_t lane = r & 31u;
+  const uint32_t dchunk = ((r >> 6) == hf) ? ((r >> 5) & 1u) : 2u;   // chunk holding the diagonal (2: none)
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     float v[32];
     tmem_ld32(taddr + c0 + 32 * i, v);
     tmem_wait_ld();
     uint32_t p[16];
+    if (dchunk == static_cast<uint32_t>(i)) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const uint32_t k = 32u * i + 2u * e;
-      const float a0 = fmaf(beta, v[2 * e], (mine && dl == k) ? diag : 0.f);
-      const float a1 = fmaf(beta, v[2 * e + 1], (mine && dl == k + 1) ? diag : 0.f);
-      p[e] = pack2_op<F>(a0, a1);
+      for (int e = 0; e < 16; ++e) {
+        const float a0 = fmaf(beta, v[2 * e], lane == 2u * e ? diag : 0.f);
+        const float a1 = fmaf(beta, v[2 * e + 1], lane == 2u * e + 1u ? diag : 0.f);
+        p[e] = pack2_op<F>(a0, a1);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) p[e] = pack2_op<F>(beta * v[2 * e], beta * v[2 * e + 1]);
     }
     tmem_st16(taddr + c0 + 16 * i, p);   // columns [c0, c0 + 32) were read before any is written
   }
@@ -503,7 +522,7 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     const float rho = (sqrtf(total) + a.eps) * a.safety;
 
     // ---- X_0 = r(M' / rho) to X_s and (packed) to D_X
-    tmem_row_to_op<F, true>(tX, tX, Xs, r, hf, 1.0f / rho);
+    tmem_row_to_op<F, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
     // M' must have left S_s before the first conversion overwrites it; that
     // conversion follows MMA1, which the issuing thread starts only after this.
     if (step_mode && gt == 0) bulk_wait_read0();
@@ -532,7 +551,8 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
       if (!bad) ++mma_seen;
       tc_fence_after();
-      tmem_row_to_op<F, true>(tP, tX, Ss, r, hf, stp->s);
+      if (stp->s == 1.f) tmem_row_to_op<F, false>(tP, tX, Ss, r, hf, 1.f);
+      else tmem_row_to_op<F, true>(tP, tX, Ss, r, hf, stp->s);
       fence_proxy_async_smem();
       tc_fence_before();
       if ((stop = group_issue<F, kJobSquare>(a, sm, g, gt, dP, stp, bad))) break;
@@ -550,7 +570,8 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       if (!bad) ++mma_seen;
       tc_fence_after();
       if (t + 1 < a.K) {
-        tmem_row_to_op<F, false>(tX, tX, Xs, r, hf, 1.f);
+        if (stp->xr == 1.f) tmem_row_to_op<F, false>(tX, tX, Xs, r, hf, 1.f);
+        else tmem_row_to_op<F, true>(tX, tX, Xs, r, hf, stp->xr);
         fence_proxy_async_smem();
         tc_fence_before();
         if ((stop = group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr, bad))) break;
@@ -585,13 +606,19 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
         for (int k = 0; k < 4; ++k) {
           const uint32_t cg = 4 * c32 + k;
           const uint32_t off = stage_off<P>(jr, rr, cg - jr * (T / 8));
-          const float *o = v + 8 * k;
-          if (a.has_o) *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(o);
+          const float *o = v + 8 * k;   // gamma_{K-1} O
+          if (a.has_o) {
+            float os[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) os[e] = a.oscale * o[e];
+            *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(os);
+          }
           if (has_w) {
+            const float lro = -a.lr * a.oscale;
             float w[8];
             unpack8(*reinterpret_cast<const uint4 *>(Ws + off), w);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = fmaf(-a.lr, o[e], w[e]);
+            for (int e = 0; e < 8; ++e) w[e] = fmaf(lro, o[e], w[e]);
             *reinterpret_cast<uint4 *>(Ws + off) = pack8_bf16(w);
           }
         }
@@ -679,20 +706,38 @@ int resident_smem_bytes() { return static_cast<int>(kSmemBytes); }
 int resident_max_smem_blocks() { return kMaxSmemBlocks; }
 
 void make_resident_steps(ResidentArgs &args, const float *coeffs, int K) {
-  // MMA2 leaves D_P = B / beta with beta = b (beta = 1 when b = 0, in which
-  // case MMA2 overwrites A with c A^2): S = r(sqrt|c / beta| A) and the sign of
-  // c / beta goes on MMA2's A operand.  MMA3 then forms r(beta D_P + a I) X.
+  // Step t with beta = b (beta = 1 when b = 0, in which case MMA2 overwrites
+  // A with c A^2) and g = sqrt|c / beta|.  The operand carries the iterate as
+  // gamma_t X_t with gamma_t = g (1 when c = 0), so MMA1 leaves
+  // D_P = gamma_t^2 A and S = r(s D_P), s = g / gamma_t^2 ... = 1 when
+  // gamma_t = g: then S S^T = g^2 gamma_t^2 A^2 and MMA2 (sign of c / beta on
+  // its A operand) leaves D_P = gamma_t^2 (A + (c / beta) A^2) = gamma_t^2 B / beta.
+  // Bop = r((beta / gamma_t^2) D_P + a I) = r(a I + B) as written, MMA3 leaves
+  // D_X = Bop gamma_t X_t = gamma_t X_{t+1}, and the next operand is
+  // r((gamma_{t+1} / gamma_t) D_X); O = D_X / gamma_{K-1}.
+  std::vector<double> gam(K);
+  for (int t = 0; t < K; ++t) {
+    const double b = coeffs[3 * t + 1], c = coeffs[3 * t + 2];
+    const double beta = (b != 0.0) ? b : 1.0;
+    const double g = sqrt(fabs(c / beta));
+    gam[t] = g > 0.0 ? g : 1.0;
+  }
   for (int t = 0; t < K; ++t) {
     const double a = coeffs[3 * t], b = coeffs[3 * t + 1], c = coeffs[3 * t + 2];
     const double beta = (b != 0.0) ? b : 1.0;
     const double ratio = c / beta;
     ResidentStep &st = args.step[t];
-    st.s = static_cast<float>(sqrt(fabs(ratio)));
+    st.s = static_cast<float>(sqrt(fabs(ratio)) / gam[t]);   // exactly 1 unless c = 0 (then 0)
+    if (sqrt(fabs(ratio)) == gam[t]) st.s = 1.f;
     st.neg2 = ratio < 0.0 ? 1u : 0u;
     st.acc2 = (b != 0.0) ? 1u : 0u;
-    st.beta = static_cast<float>(beta);
+    st.beta = static_cast<float>(beta / (gam[t] * gam[t]));
     st.a = static_cast<float>(a);
+    st.xr = t + 1 < K ? static_cast<float>(gam[t + 1] / gam[t]) : 1.f;
+    if (t + 1 < K && gam[t + 1] == gam[t]) st.xr = 1.f;
   }
+  args.gamma0 = K > 0 ? static_cast<float>(gam[0]) : 1.f;
+  args.oscale = K > 0 ? static_cast<float>(1.0 / gam[K - 1]) : 1.f;
 }
 
 template <int F, int P>

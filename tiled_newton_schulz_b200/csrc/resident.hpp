@@ -11,11 +11,13 @@ namespace himuon {
 constexpr int kMaxSteps = 16;
 
 // Per-step scalars derived on the host from (a_t, b_t, c_t); see
-// make_resident_steps() for their meaning.
+// make_resident_steps() for their meaning.  The iterate is carried scaled,
+// as gamma_t X_t, so that S needs no scaling of its own (s = 1).
 struct ResidentStep {
-  float s;          // S = r(s * A) feeds MMA2
+  float s;          // S = r(s * D_P) feeds MMA2
   float beta;       // Bop = r(beta * D_P + a * I) feeds MMA3
   float a;          // a_t
+  float xr;         // next operand r(xr * D_X) = gamma_{t+1} X_{t+1}  (xr = gamma_{t+1} / gamma_t)
   uint32_t neg2;    // MMA2 negates its A operand (c_t / beta < 0)
   uint32_t acc2;    // MMA2 accumulates onto A (b_t != 0)
 };
@@ -33,6 +35,8 @@ struct ResidentArgs {
   int32_t pack;     // tiles per 128 x 128 super-tile: 1 (T = 128), 2 (T = 64) or 4 (T = 32)
   int32_t test_stall;  // self-test: CTA 0 waits on a barrier nothing arrives on (timeout path)
   float mu, lr, eps, safety;
+  float gamma0;     // X_0 operand = r(gamma0 M' / rho)
+  float oscale;     // O = oscale * D_X after the last step (1 / gamma_{K-1})
   ResidentStep step[kMaxSteps];
   int *status;
 };
