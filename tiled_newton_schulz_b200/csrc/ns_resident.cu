@@ -521,7 +521,7 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       if (P == 1 || (32u * (w & 3)) / T == jr) total += sm.red(g)[w];
     const float rho = (sqrtf(total) + a.eps) * a.safety;
 
-    // ---- X_0 = r(M' / rho) to X_s and (packed) to D_X
+    // ---- operand g_0 X_0 = r(g_0 M' / rho) to X_s and (packed) to D_X
     tmem_row_to_op<F, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
     // M' must have left S_s before the first conversion overwrites it; that
     // conversion follows MMA1, which the issuing thread starts only after this.
@@ -547,7 +547,7 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     bool stop = false;
     for (int t = 0; t < a.K && !stop; ++t) {
       const ResidentStep *stp = &a.step[t];
-      // after MMA1: S = r(s A) to S_s and (packed) to D_X
+      // after MMA1: S = r(s D_P) (s = 1 unless c = 0) to S_s and (packed) to D_X
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
       if (!bad) ++mma_seen;
       tc_fence_after();
@@ -557,7 +557,7 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       tc_fence_before();
       if ((stop = group_issue<F, kJobSquare>(a, sm, g, gt, dP, stp, bad))) break;
       ++mma_armed;
-      // after MMA2: Bop = r(beta D_P + a I), packed in D_P
+      // after MMA2: Bop = r(beta D_P + a I) (beta = b / g^2), packed in D_P
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
       if (!bad) ++mma_seen;
       tc_fence_after();
@@ -565,7 +565,7 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       tc_fence_before();
       if ((stop = group_issue<F, kJobUpdate>(a, sm, g, gt, dP, stp, bad))) break;
       ++mma_armed;
-      // after MMA3: next operand X_t = r(D_X)
+      // after MMA3: next operand r(xr D_X) = g_{t+1} X_{t+1} (xr = 1 for constant coefficients)
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
       if (!bad) ++mma_seen;
       tc_fence_after();
