@@ -571,6 +571,7 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       na.x16_dtype = dt16;
       na.partial = pk.partial;
       na.parts = pk.parts;
+      na.keep32 = (f32 || gram) ? 1 : 0;   // the 16-bit NS path reads only the 16-bit copy
       na.eps = p.eps;
       na.safety = safety;
       HIMUON_TRY(launch_normalize(na, stream));
@@ -586,19 +587,24 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
           // A = X X^T
           rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, epi(1.f, 0.f, nullptr, a32, a16, dt16));
           if (rc) break;
-          // B' = b A + c A A + (a - 1) I
+          // 16-bit operands: Bop = r(b A + c A A + a I), and X <- r(Bop X) (fp32
+          // accumulation, the whole update in one product, as on chip).
+          // fp32: B' = b A + c A A + (a - 1) I, and X <- X + B' X on the fp32 master.
           Epilogue e2 = epi(cc, b, a32, f32 ? static_cast<float *>(bop) : nullptr, f32 ? nullptr : bop, dt16);
-          e2.diag = a - 1.f;
+          e2.diag = f32 ? a - 1.f : a;
           rc = ops.mm(f32 ? static_cast<void *>(a32) : a16, n, n, f32 ? static_cast<void *>(a32) : a16, n, n, 0, n, n,
                       n, bc, e2);
           if (rc) break;
-          // X = a X + B X = X + B' X  (fp32 master in place; operand copy ping-pongs)
+          // X = a X + B X
           if (f32) {
             rc = ops.mm(bop, n, n, x32[cur], n, m, 0, n, m, n, bc, epi(1.f, 1.f, x32[cur], x32[1 - cur], nullptr, dt16));
             cur = 1 - cur;
             xfinal = x32[cur];
           } else {
-            rc = ops.mm(bop, n, n, x16[cur], n, m, 0, n, m, n, bc, epi(1.f, 1.f, x32[0], x32[0], x16[1 - cur], dt16));
+            // the 16-bit operand for the next step, or the fp32 result after the last
+            const bool last = t + 1 == p.steps;
+            rc = ops.mm(bop, n, n, x16[cur], n, m, 0, n, m, n, bc,
+                        epi(1.f, 0.f, nullptr, last ? x32[0] : nullptr, last ? nullptr : x16[1 - cur], dt16));
             cur = 1 - cur;
           }
         }

@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(256) normalize_kernel(const NormArgs a) {
   const int64_t e0 = blockIdx.x * per, e1 = min(a.elems, e0 + per);
   for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
     const float v = x[e] * inv;
-    x[e] = v;
+    if (a.keep32) x[e] = v;
     if (a.x16) st_elem(a.x16, a.x16_dtype, t * a.elems + e, v);
   }
 }

@@ -61,6 +61,7 @@ struct NormArgs {
   int32_t x16_dtype;
   const float *partial;
   int32_t parts;
+  int32_t keep32;         // also write the normalised fp32 iterate back to x32
   float eps, safety;
 };
 cudaError_t launch_normalize(const NormArgs &a, cudaStream_t stream);
