@@ -523,6 +523,11 @@ Epilogue epi(float alpha, float beta, const float *c32, float *out32, void *out1
   e.out16 = out16;
   e.out16_dtype = dt;
   e.diag = 0.f;
+  e.sym = 0;
+  return e;
+}
+Epilogue sym(Epilogue e) {
+  e.sym = 1;
   return e;
 }
 
@@ -585,13 +590,14 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
         for (int t = 0; t < p.steps && rc == HIMUON_OK; ++t) {
           const float a = p.coeffs[3 * t], b = p.coeffs[3 * t + 1], cc = p.coeffs[3 * t + 2];
           // A = X X^T
-          rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, epi(1.f, 0.f, nullptr, a32, a16, dt16));
+          rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, sym(epi(1.f, 0.f, nullptr, a32, a16, dt16)));
           if (rc) break;
           // 16-bit operands: Bop = r(b A + c A A + a I), and X <- r(Bop X) (fp32
           // accumulation, the whole update in one product, as on chip).
           // fp32: B' = b A + c A A + (a - 1) I, and X <- X + B' X on the fp32 master.
           Epilogue e2 = epi(cc, b, a32, f32 ? static_cast<float *>(bop) : nullptr, f32 ? nullptr : bop, dt16);
           e2.diag = f32 ? a - 1.f : a;
+          e2.sym = 1;
           rc = ops.mm(f32 ? static_cast<void *>(a32) : a16, n, n, f32 ? static_cast<void *>(a32) : a16, n, n, 0, n, n,
                       n, bc, e2);
           if (rc) break;
@@ -609,7 +615,12 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
           }
         }
       } else {
-        // Gram NS (Algorithm 3): R = X X^T, Q = I; restarts X <- Q X
+        // Gram NS (Algorithm 3): R = X X^T, Q = I; restarts X <- Q X.  The terms
+        // a Q, a R, a RZ stay fp32 (C operands): folding a I into a 16-bit Z
+        // loses R's small eigen-directions below fp16's normal range.  Between
+        // restarts every n x n matrix here is a polynomial in one R, so all of
+        // them commute and every n x n product is symmetric: computed as its
+        // lower triangle.
         float *r32 = a32, *q32 = reinterpret_cast<float *>(W + L.q32), *z32 = reinterpret_cast<float *>(W + L.z32);
         float *rz32 = reinterpret_cast<float *>(W + L.rz32);
         float *q32b = f32 ? reinterpret_cast<float *>(W + L.b32) : nullptr;
@@ -622,7 +633,7 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
         auto rzop = [&]() -> void * { return f32 ? static_cast<void *>(rz32) : rz16; };
         auto qop = [&](int i) -> void * { return f32 ? static_cast<void *>(qf[i]) : q16[i]; };
         bool q_identity = true;
-        rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, epi(1.f, 0.f, nullptr, r32, r16, dt16));
+        rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, sym(epi(1.f, 0.f, nullptr, r32, r16, dt16)));
         for (int t = 1; t <= p.steps && rc == HIMUON_OK; ++t) {
           const float a = p.coeffs[3 * (t - 1)], b = p.coeffs[3 * (t - 1) + 1], cc = p.coeffs[3 * (t - 1) + 2];
           bool restart = false;
@@ -638,13 +649,13 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
                 cur = 1 - cur;
               }
               if (rc) break;
-              rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, epi(1.f, 0.f, nullptr, r32, r16, dt16));
+              rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, sym(epi(1.f, 0.f, nullptr, r32, r16, dt16)));
               if (rc) break;
             }
             q_identity = true;
           }
           // Z = b R + c R^2
-          rc = ops.mm(rop(), n, n, rop(), n, n, 0, n, n, n, bc, epi(cc, b, r32, z32, z16, dt16));
+          rc = ops.mm(rop(), n, n, rop(), n, n, 0, n, n, n, bc, sym(epi(cc, b, r32, z32, z16, dt16)));
           if (rc) break;
           // Q <- Q Z + a Q
           if (q_identity) {
@@ -652,16 +663,16 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
             q_identity = false;
           } else {
             rc = ops.mm(qop(qc), n, n, zop(), n, n, 0, n, n, n, bc,
-                        epi(1.f, a, qf[qc], qf[1 - qc], f32 ? nullptr : q16[1 - qc], dt16));
+                        sym(epi(1.f, a, qf[qc], qf[1 - qc], f32 ? nullptr : q16[1 - qc], dt16)));
             qc = 1 - qc;
             if (rc) break;
           }
           if (t == p.steps) break;   // R_K is never used
           // RZ <- R Z + a R
-          rc = ops.mm(rop(), n, n, zop(), n, n, 0, n, n, n, bc, epi(1.f, a, r32, rz32, rz16, dt16));
+          rc = ops.mm(rop(), n, n, zop(), n, n, 0, n, n, n, bc, sym(epi(1.f, a, r32, rz32, rz16, dt16)));
           if (rc) break;
           // R <- Z RZ + a RZ
-          rc = ops.mm(zop(), n, n, rzop(), n, n, 0, n, n, n, bc, epi(1.f, a, rz32, r32, r16, dt16));
+          rc = ops.mm(zop(), n, n, rzop(), n, n, 0, n, n, n, bc, sym(epi(1.f, a, rz32, r32, r16, dt16)));
         }
         if (rc == HIMUON_OK) {
           // output Q X

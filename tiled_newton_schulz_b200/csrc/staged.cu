@@ -143,13 +143,18 @@ struct EpiArgs {
   float *out32;
   void *out16;
   int32_t out16_dtype;
+  int32_t sym;      // lower-triangle tiles only, off-diagonal ones mirrored
   int64_t N;        // columns of the output matrices
   int64_t stride;   // elements per output matrix (M * N)
 };
 
 // Write 8 consecutive outputs starting at element index `o` of the batch;
-// they sit in row `row`, columns col..col+7 of their matrix.
-__device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t row, int64_t col, const float *acc) {
+// they sit in row `row`, columns col..col+7 of their matrix.  With `mirror`
+// (an off-diagonal tile of a symmetric product) they also go to rows
+// col..col+7, column `row` (element index `om` for the first; a warp's lanes
+// hold consecutive rows, so each of these scalar stores is coalesced).
+__device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t row, int64_t col, const float *acc,
+                                           bool mirror = false, int64_t om = 0) {
   float v[8];
   if (e.c32) {
     const float4 c0 = *reinterpret_cast<const float4 *>(e.c32 + o);
@@ -168,6 +173,10 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
   if (e.out32) {
     *reinterpret_cast<float4 *>(e.out32 + o) = make_float4(v[0], v[1], v[2], v[3]);
     *reinterpret_cast<float4 *>(e.out32 + o + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    if (mirror) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) e.out32[om + i * e.N] = v[i];
+    }
   }
   if (e.out16) {
     uint4 u;
@@ -181,6 +190,12 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
 #pragma unroll
       for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
       *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(e.out16) + o) = u;
+    }
+    if (mirror) {
+      const uint16_t *hs = reinterpret_cast<const uint16_t *>(&u);
+      uint16_t *d = static_cast<uint16_t *>(e.out16);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[om + i * e.N] = hs[i];
     }
   }
 }
@@ -209,7 +224,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *done = empty + kStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int32_t n0 = blockIdx.x * 128, m0 = blockIdx.y * 128, z = blockIdx.z;
+  int32_t n0 = blockIdx.x * 128, m0 = blockIdx.y * 128;
+  const int32_t z = blockIdx.z;
+  if (a.ep.sym) {   // blockIdx.x enumerates the tiles (ti, tj), tj <= ti, row by row
+    const int32_t k = blockIdx.x;
+    int32_t ti = static_cast<int32_t>((sqrtf(8.f * k + 1.f) - 1.f) * 0.5f);
+    while ((ti + 1) * (ti + 2) / 2 <= k) ++ti;
+    while (ti * (ti + 1) / 2 > k) --ti;
+    m0 = ti * 128;
+    n0 = (k - ti * (ti + 1) / 2) * 128;
+  }
+  const bool mirror = a.ep.sym && m0 != n0;
   const int nk = static_cast<int>(a.K / 64);
 
   if (threadIdx.x == 0) {
@@ -274,7 +299,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(taddr + 32 * i, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) epi_store8(a.ep, obase + 32 * i + 8 * j, m0 + row, n0 + 32 * i + 8 * j, v + 8 * j);
+        for (int j = 0; j < 4; ++j) {
+          const int64_t col = n0 + 32 * i + 8 * j;
+          epi_store8(a.ep, obase + 32 * i + 8 * j, m0 + row, col, v + 8 * j, mirror,
+                     z * a.ep.stride + col * a.ep.N + m0 + row);
+        }
       }
     }
   }
@@ -381,6 +410,7 @@ EpiArgs to_epi(const Epilogue &e, int64_t M, int64_t N) {
   a.out32 = e.out32;
   a.out16 = e.out16;
   a.out16_dtype = e.out16_dtype;
+  a.sym = e.sym && M == N;
   a.N = N;
   a.stride = M * N;
   return a;
@@ -404,6 +434,10 @@ cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int6
   a.ep = to_epi(ep, M, N);
   a.status = status;
   dim3 grid(static_cast<unsigned>(N / 128), static_cast<unsigned>(M / 128), static_cast<unsigned>(batch));
+  if (a.ep.sym) {
+    const int64_t nt = M / 128;
+    grid = dim3(static_cast<unsigned>(nt * (nt + 1) / 2), 1, static_cast<unsigned>(batch));
+  }
   cudaError_t e;
   if (b_trans) {
     e = cudaFuncSetAttribute(gemm_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);

@@ -27,6 +27,10 @@ struct Epilogue {
   float *out32;
   void *out16;
   int32_t out16_dtype;
+  // The product is symmetric (M == N; and c32, if given, symmetric): the
+  // tensor-core version computes only the 128 x 128 tiles on and below the
+  // diagonal and writes each off-diagonal one twice, mirrored.
+  int32_t sym;
 };
 
 // acc = A * B^T (b_trans = 1, B is N x K) or A * B (b_trans = 0, B is K x N),
