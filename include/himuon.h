@@ -140,7 +140,10 @@ HIMUON_API int himuon_ns_full(const himuon_mat *in, const himuon_mat *out, int32
  * Q <- I at the steps in p->restart_at) Z = b R + c R^2, Q <- Q Z + a Q,
  * RZ <- R Z + a R, R <- Z RZ + a RZ; output Q X (transposed back).
  * Equal to himuon_ns_full in exact arithmetic.  compute: FP16 (the page's
- * advice for this variant), BF16 or FP32.  p->tile is ignored.
+ * advice for this variant), BF16 or FP32.  p->tile = 0 (or any T at least as
+ * large as a block's sides) runs it on the whole (split block of the) matrix;
+ * a smaller T applies it to each T x T tile ("Hierarchical Muon" abstract:
+ * the same map per tile, ragged edge tiles smaller), on the staged path.
  */
 HIMUON_API int himuon_gram_ns(const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,
                    const himuon_ns_params *p, void *ws, size_t ws_bytes, void *stream);

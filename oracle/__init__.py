@@ -124,6 +124,21 @@ def gram_ns(x, coeffs, K: int | None = None, restart: Sequence[int] = (3,), eps:
     return out
 
 
+def gram_ns_tiled(x, T: int, coeffs, K: int | None = None, restart: Sequence[int] = (3,),
+                  eps: float = EPS) -> np.ndarray:
+    """Gram NS applied to each T x T tile ("Hierarchical Muon" abstract: the
+    same map per tile, reassembled; ragged edge tiles smaller).  T <= 0 or at
+    least the matrix's sides: the whole matrix."""
+    X = _f64(x)
+    H, W = X.shape
+    if T <= 0 or T >= max(H, W):
+        return gram_ns(X, coeffs, K, restart, eps)
+    out = np.zeros((H, W), dtype=np.float64)
+    for r0, c0, h, w in tile_grid(H, W, T):
+        out[r0:r0 + h, c0:c0 + w] = gram_ns(X[r0:r0 + h, c0:c0 + w], coeffs, K, restart, eps)
+    return out
+
+
 def split_blocks(shape: tuple[int, int], split: tuple[int, Sequence[int]] | None):
     """CMuon split: list of (row0, col0, rows, cols) blocks of a fused matrix.
 

@@ -227,6 +227,25 @@ def test_gram_ns_fp16(hm, restart):
     assert max_sv_diff(yy, ref, 0) <= SVTOL
 
 
+@pytest.mark.parametrize("T", [128, 256])
+def test_gram_ns_tiled_fp16(hm, T):
+    """Gram NS applied per tile (ragged edge rows and columns), fp16 operands,
+    restart at t = 3, against the oracle's tile-by-tile Gram NS."""
+    H, W = 640, 832
+    X = inputs.low_rank_plus_noise(H, W, inputs.sigma_exp(H, 32.0), 1e-3, seed=12)
+    x = dev(X, torch.bfloat16)
+    y = torch.empty_like(x)
+    hm.gram_ns([x], [y], hm.params(T, QUINTIC, steps=5, compute=hm.FP16, restart=(3,)))
+    assert hm.device_status() == 0
+    xin = to_np(x)
+    ref = oracle.gram_ns_tiled(xin, T, C32, restart=(3,))
+    yy = to_np(y)
+    for r0, c0, h, w in oracle.tile_grid(H, W, T):
+        sl = np.s_[r0:r0 + h, c0:c0 + w]
+        assert np.linalg.norm(yy[sl] - ref[sl]) / np.linalg.norm(ref[sl]) <= TOL16
+        assert max_sv_diff(yy[sl], ref[sl], 0) <= SVTOL
+
+
 def test_split_qkv_blocks(hm):
     """A fused 256 x 768 tensor split into three 256 x 256 blocks before full NS."""
     X = inputs.gaussian((256, 768), seed=31)

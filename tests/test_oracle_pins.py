@@ -172,6 +172,23 @@ def test_gram_ns_on_low_rank_spectrum():
     assert rel(oracle.gram_ns(X, CFG * 5, restart=(3,)), ns_by_svd(X, CFG * 5)) < 1e-10
 
 
+@pytest.mark.parametrize("T", [8, 16, 40])
+def test_gram_ns_tiled_is_tilewise_svd_map(T):
+    """Tiled Gram NS: each tile (ragged edges included, tall ones too) is
+    mapped by the SVD closed form of its own NS polynomial, independently of
+    its neighbours: a tile scaled by 1000 changes no other tile."""
+    X = inputs.gaussian((50, 70), seed=T)
+    g = oracle.gram_ns_tiled(X, T, C5, restart=(3,))
+    for r0, c0, h, w in oracle.tile_grid(50, 70, T):
+        assert rel(g[r0:r0 + h, c0:c0 + w], ns_by_svd(X[r0:r0 + h, c0:c0 + w], C5)) < 1e-10
+    Y = X.copy()
+    Y[:T, :T] *= 1000.0
+    gy = oracle.gram_ns_tiled(Y, T, C5, restart=(3,))
+    assert np.array_equal(gy[T:, :], g[T:, :]) and np.array_equal(gy[:T, T:], g[:T, T:])
+    assert rel(gy[:T, :T], g[:T, :T]) < 1e-7           # scale-invariant up to the eps in the norm
+    assert rel(oracle.gram_ns_tiled(X, 0, C5), oracle.gram_ns(X, C5)) == 0.0
+
+
 def test_momentum_step_closed_form():
     rng = np.random.default_rng(9)
     W, M, G = (rng.standard_normal((6, 9)) for _ in range(3))

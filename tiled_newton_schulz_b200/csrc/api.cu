@@ -289,7 +289,7 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
                std::shared_ptr<Plan> &out) {
   auto plan = std::make_shared<Plan>();
   plan->device = device;
-  int rc = make_blocks(cm, splits, op == HIMUON_OP_NS_FULL || op == HIMUON_OP_GRAM_NS ? 0 : p.tile, plan->blocks,
+  int rc = make_blocks(cm, splits, op == HIMUON_OP_NS_FULL ? 0 : p.tile, plan->blocks,
                        &plan->n_tiles);
   if (rc) return rc;
   const int pack = op != HIMUON_OP_GRAM_NS ? resident_pack(cm, plan->blocks, p) : 0;
@@ -922,7 +922,7 @@ int64_t himuon_workspace_size(const himuon_mat *mats, int32_t n, const himuon_sp
   if (rc) return rc;
   std::vector<HostBlock> blocks;
   int64_t n_tiles = 0;
-  const int64_t tile = (op == HIMUON_OP_NS_FULL || op == HIMUON_OP_GRAM_NS) ? 0 : p->tile;
+  const int64_t tile = op == HIMUON_OP_NS_FULL ? 0 : p->tile;
   rc = make_blocks(cm, splits, tile, blocks, &n_tiles);
   if (rc) return rc;
   if (op != HIMUON_OP_GRAM_NS && resident_pack(cm, blocks, *p) > 0) return 0;
