@@ -60,22 +60,23 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
   float *x = a.x32 + t * a.n * a.m;
   float ss = 0.f;
   if (i0 < i1) {
-    const int64_t cnt = static_cast<int64_t>(i1 - i0) * tl.w;
     const void *src = b.ptr[kRoleIn];
     const int64_t ld = b.ld[kRoleIn];
     const int32_t dt = b.dtype[kRoleIn];
-    for (int64_t e = threadIdx.x; e < cnt; e += blockDim.x) {
-      const int32_t i = i0 + static_cast<int32_t>(e / tl.w), j = static_cast<int32_t>(e % tl.w);
-      const int64_t gi = static_cast<int64_t>(tl.r0 + i) * ld + tl.c0 + j;
-      float v = ld_elem(src, dt, gi);
-      if (a.mode == 1) {
-        const float g = ld_elem(b.ptr[kRoleG], b.dtype[kRoleG], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleG] + tl.c0 + j);
-        v = fmaf(a.mu, v, g);
-        st_elem(b.ptr[kRoleIn], dt, gi, v);
+    for (int32_t i = i0; i < i1; ++i) {
+      for (int32_t j = threadIdx.x; j < tl.w; j += blockDim.x) {
+        const int64_t gi = static_cast<int64_t>(tl.r0 + i) * ld + tl.c0 + j;
+        float v = ld_elem(src, dt, gi);
+        if (a.mode == 1) {
+          const float g =
+              ld_elem(b.ptr[kRoleG], b.dtype[kRoleG], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleG] + tl.c0 + j);
+          v = fmaf(a.mu, v, g);
+          st_elem(b.ptr[kRoleIn], dt, gi, v);
+        }
+        ss = fmaf(v, v, ss);
+        const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
+        x[xo] = v;
       }
-      ss = fmaf(v, v, ss);
-      const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
-      x[xo] = v;
     }
   }
   const float s = block_sum<256>(ss, scratch);
@@ -106,17 +107,17 @@ __global__ void __launch_bounds__(256) unpack_kernel(const UnpackArgs a, int32_t
   const int32_t i0 = blockIdx.x * rows_per_part, i1 = min(tl.h, i0 + rows_per_part);
   if (i0 >= i1) return;
   const float *x = a.x32 + t * a.n * a.m;
-  const int64_t cnt = static_cast<int64_t>(i1 - i0) * tl.w;
-  for (int64_t e = threadIdx.x; e < cnt; e += blockDim.x) {
-    const int32_t i = i0 + static_cast<int32_t>(e / tl.w), j = static_cast<int32_t>(e % tl.w);
-    const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
-    const float o = x[xo];
-    if (b.ptr[kRoleOut])
-      st_elem(b.ptr[kRoleOut], b.dtype[kRoleOut], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleOut] + tl.c0 + j, o);
-    if (a.mode == 1 && b.ptr[kRoleW]) {
-      const int64_t gi = static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleW] + tl.c0 + j;
-      const float w = ld_elem(b.ptr[kRoleW], b.dtype[kRoleW], gi);
-      st_elem(b.ptr[kRoleW], b.dtype[kRoleW], gi, fmaf(-a.lr, o, w));
+  for (int32_t i = i0; i < i1; ++i) {
+    for (int32_t j = threadIdx.x; j < tl.w; j += blockDim.x) {
+      const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
+      const float o = x[xo];
+      if (b.ptr[kRoleOut])
+        st_elem(b.ptr[kRoleOut], b.dtype[kRoleOut], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleOut] + tl.c0 + j, o);
+      if (a.mode == 1 && b.ptr[kRoleW]) {
+        const int64_t gi = static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleW] + tl.c0 + j;
+        const float w = ld_elem(b.ptr[kRoleW], b.dtype[kRoleW], gi);
+        st_elem(b.ptr[kRoleW], b.dtype[kRoleW], gi, fmaf(-a.lr, o, w));
+      }
     }
   }
 }
@@ -201,9 +202,11 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
 }
 
 // ---------------------------------------------------------------- tcgen05 GEMM
-constexpr int kStages = 3;
+// Pipeline depth: 3 stages for long K; 2 when K <= 256 (at most 4 k-blocks),
+// which lets 3 CTAs share an SM and hide each other's latency.
 constexpr uint32_t kStageA = 16384, kStageB = 16384, kStageBytes = kStageA + kStageB;
-constexpr uint32_t kGemmSmem = kStages * kStageBytes + 128 + 1024;
+template <int STAGES>
+constexpr uint32_t gemm_smem() { return STAGES * kStageBytes + 128 + 1024; }
 constexpr int kGemmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 
 struct GemmTcArgs {
@@ -213,7 +216,7 @@ struct GemmTcArgs {
   int *status;
 };
 
-template <int B_MN>
+template <int B_MN, int kStages>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const GemmTcArgs a) {
@@ -439,17 +442,17 @@ cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int6
     grid = dim3(static_cast<unsigned>(nt * (nt + 1) / 2), 1, static_cast<unsigned>(batch));
   }
   cudaError_t e;
-  if (b_trans) {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-    if (e != cudaSuccess) return e;
+  auto go = [&](auto kern, uint32_t smem) -> cudaError_t {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
     count_launch();
-    gemm_tc_kernel<0><<<grid, kGemmThreads, kGemmSmem, stream>>>(ma, mb, a);
-  } else {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-    if (e != cudaSuccess) return e;
-    count_launch();
-    gemm_tc_kernel<1><<<grid, kGemmThreads, kGemmSmem, stream>>>(ma, mb, a);
-  }
+    kern<<<grid, kGemmThreads, smem, stream>>>(ma, mb, a);
+    return cudaSuccess;
+  };
+  const bool short_k = K <= 256;
+  if (b_trans) e = short_k ? go(gemm_tc_kernel<0, 2>, gemm_smem<2>()) : go(gemm_tc_kernel<0, 3>, gemm_smem<3>());
+  else e = short_k ? go(gemm_tc_kernel<1, 2>, gemm_smem<2>()) : go(gemm_tc_kernel<1, 3>, gemm_smem<3>());
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
