@@ -132,11 +132,6 @@ __global__ void add_identity_kernel(const float *z, float a, float *q32, void *q
   }
 }
 
-__global__ void to16_kernel(const float *x, void *y, int32_t dt, int64_t total) {
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x)
-    st_elem(y, dt, e, x[e]);
-}
-
 // ---------------------------------------------------------------- epilogue
 struct EpiArgs {
   float alpha, beta, diag;
@@ -500,13 +495,6 @@ cudaError_t launch_add_identity(const float *z32, float a, float *q32, void *q16
   const int blocks = static_cast<int>((total + 255) / 256 < 65535 ? (total + 255) / 256 : 65535);
   count_launch();
   add_identity_kernel<<<blocks, 256, 0, stream>>>(z32, a, q32, q16, q16_dtype, n, total);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_to16(const float *x32, void *x16, int32_t dtype, int64_t count, cudaStream_t stream) {
-  const int blocks = static_cast<int>((count + 255) / 256 < 65535 ? (count + 255) / 256 : 65535);
-  count_launch();
-  to16_kernel<<<blocks, 256, 0, stream>>>(x32, x16, dtype, count);
   return cudaGetLastError();
 }
 

@@ -84,7 +84,5 @@ cudaError_t launch_unpack(const UnpackArgs &a, cudaStream_t stream);
 // q32/q16 <- z32 + a I  (n x n per matrix); used when Q = I in Gram NS
 cudaError_t launch_add_identity(const float *z32, float a, float *q32, void *q16, int32_t q16_dtype, int64_t n,
                                 int64_t batch, cudaStream_t stream);
-// 16-bit copy of an fp32 batch
-cudaError_t launch_to16(const float *x32, void *x16, int32_t dtype, int64_t count, cudaStream_t stream);
 
 }  // namespace himuon
