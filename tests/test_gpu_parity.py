@@ -91,6 +91,62 @@ def test_resident_tiled_ns(hm, H, W, compute):
     check16(y, oracle.ns_tiled(xin, 128, C32), 128, bf16=compute == "bf16")
 
 
+# Step lists for the on-chip kernel's scaled operand: the pages' quintic step,
+# the textbook cubic Newton-Schulz step (c = 0: the operand is not rescaled and
+# S is zero) and an odd quintic with b = 0 (MMA2 overwrites instead of
+# accumulating); mixing them makes the operand scale change between steps.
+QUINTIC_T = tuple(QUINTIC)
+CUBIC = (1.5, -0.5, 0.0)
+NO_B = (1.5, 0.0, -0.5)
+# Sixteen steps (the maximum) end in cubic steps, which contract towards the
+# polar factor: sixteen quintic steps do not contract, and their bf16 operand
+# roundings add up past the 3e-2 budget (an emulation of exactly the kernel's
+# rounding points gives 5.2% bf16 / 3.1% fp16 per tile for them, 2.3% / 0.5%
+# for this list; the GPU matched the emulation).
+STEP_LISTS = {
+    "K1": [QUINTIC_T],
+    "K16": [QUINTIC_T] * 5 + [CUBIC] * 11,
+    "mixed": [QUINTIC_T, CUBIC, NO_B, (2.0, -1.5, 0.5), QUINTIC_T, CUBIC],
+}
+
+
+@pytest.mark.parametrize("compute", ["bf16", "fp16"])
+@pytest.mark.parametrize("T", [128, 64])
+@pytest.mark.parametrize("steps", sorted(STEP_LISTS))
+def test_resident_step_lists(hm, steps, T, compute):
+    """One step, the maximum of sixteen, and a list whose coefficients change
+    from step to step (including c = 0 and b = 0), on the on-chip kernel."""
+    X = inputs.low_rank_plus_noise(256, 384, inputs.sigma_inverse(32), 0.01, seed=T + len(steps))
+    co = STEP_LISTS[steps]
+    x = dev(X, torch.bfloat16)
+    y = torch.empty_like(x)
+    hm.ns_tiled([x], [y], hm.params(T, co, compute=hm.BF16 if compute == "bf16" else hm.FP16))
+    assert hm.device_status() == 0
+    c32 = [tuple(float(np.float32(v)) for v in tri) for tri in co]
+    check16(to_np(y), oracle.ns_tiled(to_np(x), T, c32), T, bf16=compute == "bf16")
+
+
+@pytest.mark.parametrize("steps", ["mixed", "K1"])
+def test_momentum_step_step_lists(hm, steps):
+    """The fused step (momentum prologue, W update and O out) with a step list
+    whose last step sets the output scale differently from the first."""
+    co = STEP_LISTS[steps]
+    H, W = 256, 384
+    w = dev(0.02 * inputs.gaussian((H, W), seed=3), torch.bfloat16)
+    m = dev(inputs.low_rank_plus_noise(H, W, inputs.sigma_inverse(16), 0.01, seed=4), torch.bfloat16)
+    g = dev(inputs.low_rank_plus_noise(H, W, inputs.sigma_inverse(16), 0.01, seed=5), torch.bfloat16)
+    o = torch.empty_like(m)
+    w0, m0, g0 = to_np(w), to_np(m), to_np(g)
+    hm.momentum_step([w], [m], [g], 0.95, 0.02, hm.params(128, co), update_out=[o])
+    assert hm.device_status() == 0
+    c32 = [tuple(float(np.float32(v)) for v in tri) for tri in co]
+    W2, M2, O = oracle.momentum_step(w0, m0, g0, 0.95, 0.02, 128, c32)
+    assert np.all(np.abs(to_np(m) - M2) <= bf16_ulp(M2))
+    check16(to_np(o), O, 128, bf16=True)
+    bound = np.linalg.norm(0.5 * bf16_ulp(W2)) + float(np.float32(0.02)) * TOL16 * np.linalg.norm(O)
+    assert np.linalg.norm(to_np(w) - W2) <= bound
+
+
 @pytest.mark.parametrize("compute", ["bf16", "fp16"])
 @pytest.mark.parametrize("T", [32, 64])
 @pytest.mark.parametrize("H,W", [(256, 384), (300, 500), (100, 70), (33, 65), (128, 4096)])
