@@ -54,6 +54,14 @@ bool log_enabled() {
   return v == 1;
 }
 
+// HIMUON_FORCE_PATH=staged sends calls that would run on chip through the
+// staged path instead (A/B comparisons of the two paths on the same call);
+// read on every call and part of the plan key.
+bool force_staged() {
+  const char *e = getenv("HIMUON_FORCE_PATH");
+  return e && strcmp(e, "staged") == 0;
+}
+
 size_t elem_size(int32_t dt) { return dt == HIMUON_FP32 ? 4 : 2; }
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
@@ -251,6 +259,8 @@ std::string plan_key(int device, int op, const CallMats &cm, const himuon_split 
   put(&cm.n, sizeof cm.n);
   put(&p.tile, sizeof p.tile);
   put(&p.compute, sizeof p.compute);
+  const int staged = force_staged() ? 1 : 0;
+  put(&staged, sizeof staged);
   for (int r = 0; r < kNumRoles; ++r) {
     const int present = cm.role[r] ? 1 : 0;
     put(&present, sizeof present);
@@ -292,7 +302,7 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
   int rc = make_blocks(cm, splits, op == HIMUON_OP_NS_FULL ? 0 : p.tile, plan->blocks,
                        &plan->n_tiles);
   if (rc) return rc;
-  const int pack = op != HIMUON_OP_GRAM_NS ? resident_pack(cm, plan->blocks, p) : 0;
+  const int pack = (op != HIMUON_OP_GRAM_NS && !force_staged()) ? resident_pack(cm, plan->blocks, p) : 0;
   const bool resident = pack > 0;
   plan->path = resident ? kPathResident : kPathStaged;
   plan->pack = resident ? pack : 1;
@@ -925,7 +935,7 @@ int64_t himuon_workspace_size(const himuon_mat *mats, int32_t n, const himuon_sp
   const int64_t tile = op == HIMUON_OP_NS_FULL ? 0 : p->tile;
   rc = make_blocks(cm, splits, tile, blocks, &n_tiles);
   if (rc) return rc;
-  if (op != HIMUON_OP_GRAM_NS && resident_pack(cm, blocks, *p) > 0) return 0;
+  if (op != HIMUON_OP_GRAM_NS && !force_staged() && resident_pack(cm, blocks, *p) > 0) return 0;
   // staged: one tile of the largest class is the minimum; a full chunk of every
   // class makes the call run in one chunk per class.
   int64_t need = 0;
