@@ -56,18 +56,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
       : "memory");
   return ok != 0;
 }
-// Non-blocking probe of the same condition (never suspends the thread).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t phase) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(phase)
-      : "memory");
-  return ok != 0;
-}
 // Bounded wait for the phase with parity `phase` to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, int *status) {
   if (mbar_try_wait(bar, phase)) return true;
@@ -83,9 +71,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, int *st
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 // Named barrier that also ORs a predicate over the participating threads:
 // every thread gets the same answer, so a group can agree to stop.
