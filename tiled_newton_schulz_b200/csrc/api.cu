@@ -573,7 +573,6 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       pk.m = m;
       pk.x32 = x32[0];
       pk.partial = reinterpret_cast<float *>(W + L.partial);
-      pk.rows_per_part = 32;
       pk.parts = static_cast<int32_t>((std::max(n, m) + 31) / 32);
       pk.mode = step ? 1 : 0;
       pk.mu = mu;

@@ -49,14 +49,17 @@ __device__ __forceinline__ float block_sum(float v, float *scratch) {
 }
 
 // ---------------------------------------------------------------- pack
-// grid (parts, tiles): CTA p copies source rows [p*rpp, (p+1)*rpp) of its tile.
+// grid (parts, tiles): CTA p copies source rows [p*rpp, (p+1)*rpp) of its
+// tile, rpp = ceil(rows / parts), so every part of a tile has work whatever
+// its orientation.
 __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
   __shared__ float scratch[8];
   const int64_t t = blockIdx.y;
   const DevTile tl = a.tiles[t];
   const DevBlock &b = a.blocks[tl.block];
-  const int32_t i0 = blockIdx.x * a.rows_per_part;
-  const int32_t i1 = min(tl.h, i0 + a.rows_per_part);
+  const int32_t rpp = (tl.h + a.parts - 1) / a.parts;
+  const int32_t i0 = blockIdx.x * rpp;
+  const int32_t i1 = min(tl.h, i0 + rpp);
   float *x = a.x32 + t * a.n * a.m;
   float ss = 0.f;
   if (i0 < i1) {
@@ -100,11 +103,12 @@ __global__ void __launch_bounds__(256) normalize_kernel(const NormArgs a) {
 }
 
 // grid (parts, tiles)
-__global__ void __launch_bounds__(256) unpack_kernel(const UnpackArgs a, int32_t rows_per_part) {
+__global__ void __launch_bounds__(256) unpack_kernel(const UnpackArgs a, int32_t parts) {
   const int64_t t = blockIdx.y;
   const DevTile tl = a.tiles[t];
   const DevBlock &b = a.blocks[tl.block];
-  const int32_t i0 = blockIdx.x * rows_per_part, i1 = min(tl.h, i0 + rows_per_part);
+  const int32_t rpp = (tl.h + parts - 1) / parts;
+  const int32_t i0 = blockIdx.x * rpp, i1 = min(tl.h, i0 + rpp);
   if (i0 >= i1) return;
   const float *x = a.x32 + t * a.n * a.m;
   for (int32_t i = i0; i < i1; ++i) {
@@ -480,12 +484,11 @@ cudaError_t launch_normalize(const NormArgs &a, cudaStream_t stream) {
 }
 
 cudaError_t launch_unpack(const UnpackArgs &a, cudaStream_t stream) {
-  const int32_t rpp = 32;
   const int64_t side = a.n > a.m ? a.n : a.m;   // a tile has at most max(n, m) rows
-  const int64_t parts = (side + rpp - 1) / rpp;
+  const int64_t parts = (side + 31) / 32;
   dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(a.n_tiles));
   count_launch();
-  unpack_kernel<<<grid, 256, 0, stream>>>(a, rpp);
+  unpack_kernel<<<grid, 256, 0, stream>>>(a, static_cast<int32_t>(parts));
   return cudaGetLastError();
 }
 

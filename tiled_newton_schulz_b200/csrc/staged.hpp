@@ -51,7 +51,6 @@ struct PackArgs {
   float *x32;             // n_tiles * n * m
   float *partial;         // n_tiles * parts
   int32_t parts;          // partial sums per tile (row slices of the source tile)
-  int32_t rows_per_part;
   int32_t mode;           // 0: NS input; 1: momentum (M' = mu M + G written back to M)
   float mu;
 };
