@@ -34,7 +34,8 @@
  *    that only the device can see (a wait that timed out, a bad descriptor)
  *    set a device status word read by himuon_get_device_status(); kernels never
  *    trap.
- *  - Not thread-safe: serialise calls from different host threads.
+ *  - Not thread-safe: serialise calls from different host threads (the plan
+ *    cache is locked internally, but the device status word is shared).
  */
 #ifndef HIMUON_H_
 #define HIMUON_H_

@@ -12,6 +12,7 @@
 #include <atomic>
 #include <list>
 #include <map>
+#include <mutex>
 #include <memory>
 #include <string>
 #include <vector>
@@ -286,6 +287,7 @@ std::string plan_key(int device, int op, const CallMats &cm, const himuon_split 
 }
 
 struct PlanCache {
+  std::mutex mu;   // lookups from several host threads do not corrupt the cache
   std::list<std::pair<std::string, std::shared_ptr<Plan>>> lru;
   std::map<std::string, std::list<std::pair<std::string, std::shared_ptr<Plan>>>::iterator> index;
   static constexpr size_t kCap = 32;
@@ -403,6 +405,7 @@ int get_plan(int op, const CallMats &cm, const himuon_split *splits, const himuo
   if (cudaGetDevice(&device) != cudaSuccess) return HIMUON_ERR_NO_DEVICE;
   const std::string key = plan_key(device, op, cm, splits, p);
   PlanCache &c = cache();
+  std::lock_guard<std::mutex> lock(c.mu);
   auto it = c.index.find(key);
   if (it != c.index.end()) {
     c.lru.splice(c.lru.begin(), c.lru, it->second);
