@@ -49,9 +49,48 @@ __device__ __forceinline__ float block_sum(float v, float *scratch) {
 }
 
 // ---------------------------------------------------------------- pack
+// 8 consecutive 16-bit values of either type, to fp32
+__device__ __forceinline__ void ld8_16(const void *p, int32_t dtype, int64_t i, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p) + i);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (dtype == HIMUON_BF16) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[k]));
+      v[2 * k] = f.x;
+      v[2 * k + 1] = f.y;
+    } else {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[k]));
+      v[2 * k] = f.x;
+      v[2 * k + 1] = f.y;
+    }
+  }
+}
+__device__ __forceinline__ void st8_16(void *p, int32_t dtype, int64_t i, const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (dtype == HIMUON_BF16) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+      w[k] = *reinterpret_cast<const uint32_t *>(&h);
+    } else {
+      const __half2 h = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+      w[k] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+  }
+  *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p) + i) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+// Runs of 8 elements of a role can be moved as one 16-byte access when the
+// role is 16-bit, its base is 16-byte aligned and its rows and the tile's
+// first column keep that alignment.
+__device__ __forceinline__ bool vec8_ok(const void *p, int32_t dtype, int64_t ld, int32_t c0) {
+  return p && dtype != HIMUON_FP32 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0 && (ld & 7) == 0 && (c0 & 7) == 0;
+}
+
 // grid (parts, tiles): CTA p copies source rows [p*rpp, (p+1)*rpp) of its
 // tile, rpp = ceil(rows / parts), so every part of a tile has work whatever
-// its orientation.
+// its orientation.  The CTA's threads run over (row, 8-column run) pairs,
+// with 16-byte accesses where the roles allow them.
 __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
   __shared__ float scratch[8];
   const int64_t t = blockIdx.y;
@@ -66,20 +105,46 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
     const void *src = b.ptr[kRoleIn];
     const int64_t ld = b.ld[kRoleIn];
     const int32_t dt = b.dtype[kRoleIn];
-    for (int32_t i = i0; i < i1; ++i) {
-      for (int32_t j = threadIdx.x; j < tl.w; j += blockDim.x) {
-        const int64_t gi = static_cast<int64_t>(tl.r0 + i) * ld + tl.c0 + j;
-        float v = ld_elem(src, dt, gi);
-        if (a.mode == 1) {
-          const float g =
-              ld_elem(b.ptr[kRoleG], b.dtype[kRoleG], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleG] + tl.c0 + j);
-          v = fmaf(a.mu, v, g);
-          st_elem(b.ptr[kRoleIn], dt, gi, v);
-        }
-        ss = fmaf(v, v, ss);
-        const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
-        x[xo] = v;
+    const void *gsrc = b.ptr[kRoleG];
+    const int64_t ldg = b.ld[kRoleG];
+    const int32_t dtg = b.dtype[kRoleG];
+    const bool vec = vec8_ok(src, dt, ld, tl.c0) && (a.mode == 0 || vec8_ok(gsrc, dtg, ldg, tl.c0));
+    const int32_t runs = vec ? tl.w / 8 : 0;            // whole 8-column runs per row
+    const int32_t rest = tl.w - 8 * runs;                // columns left to the scalar loop
+    const int32_t rows = i1 - i0;
+    for (int32_t k = threadIdx.x; k < rows * runs; k += blockDim.x) {
+      const int32_t i = i0 + k / runs, j = 8 * (k % runs);
+      const int64_t gi = static_cast<int64_t>(tl.r0 + i) * ld + tl.c0 + j;
+      float v[8];
+      ld8_16(src, dt, gi, v);
+      if (a.mode == 1) {
+        float g[8];
+        ld8_16(gsrc, dtg, static_cast<int64_t>(tl.r0 + i) * ldg + tl.c0 + j, g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = fmaf(a.mu, v[e], g[e]);
+        st8_16(b.ptr[kRoleIn], dt, gi, v);
       }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+      if (tl.transposed) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[static_cast<int64_t>(j + e) * a.m + i] = v[e];
+      } else {
+        float4 *xo = reinterpret_cast<float4 *>(x + static_cast<int64_t>(i) * a.m + j);
+        xo[0] = make_float4(v[0], v[1], v[2], v[3]);
+        xo[1] = make_float4(v[4], v[5], v[6], v[7]);
+      }
+    }
+    for (int32_t k = threadIdx.x; k < rows * rest; k += blockDim.x) {
+      const int32_t i = i0 + k / rest, j = 8 * runs + k % rest;
+      const int64_t gi = static_cast<int64_t>(tl.r0 + i) * ld + tl.c0 + j;
+      float v = ld_elem(src, dt, gi);
+      if (a.mode == 1) {
+        v = fmaf(a.mu, v, ld_elem(gsrc, dtg, static_cast<int64_t>(tl.r0 + i) * ldg + tl.c0 + j));
+        st_elem(b.ptr[kRoleIn], dt, gi, v);
+      }
+      ss = fmaf(v, v, ss);
+      x[tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j] = v;
     }
   }
   const float s = block_sum<256>(ss, scratch);
@@ -102,7 +167,8 @@ __global__ void __launch_bounds__(256) normalize_kernel(const NormArgs a) {
   }
 }
 
-// grid (parts, tiles)
+// grid (parts, tiles), rows split as in pack_kernel; 8-column runs where the
+// roles allow 16-byte accesses.
 __global__ void __launch_bounds__(256) unpack_kernel(const UnpackArgs a, int32_t parts) {
   const int64_t t = blockIdx.y;
   const DevTile tl = a.tiles[t];
@@ -111,17 +177,43 @@ __global__ void __launch_bounds__(256) unpack_kernel(const UnpackArgs a, int32_t
   const int32_t i0 = blockIdx.x * rpp, i1 = min(tl.h, i0 + rpp);
   if (i0 >= i1) return;
   const float *x = a.x32 + t * a.n * a.m;
-  for (int32_t i = i0; i < i1; ++i) {
-    for (int32_t j = threadIdx.x; j < tl.w; j += blockDim.x) {
-      const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
-      const float o = x[xo];
-      if (b.ptr[kRoleOut])
-        st_elem(b.ptr[kRoleOut], b.dtype[kRoleOut], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleOut] + tl.c0 + j, o);
-      if (a.mode == 1 && b.ptr[kRoleW]) {
-        const int64_t gi = static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleW] + tl.c0 + j;
-        const float w = ld_elem(b.ptr[kRoleW], b.dtype[kRoleW], gi);
-        st_elem(b.ptr[kRoleW], b.dtype[kRoleW], gi, fmaf(-a.lr, o, w));
-      }
+  void *out = b.ptr[kRoleOut];
+  void *wp = a.mode == 1 ? b.ptr[kRoleW] : nullptr;
+  const bool vec = (!out || vec8_ok(out, b.dtype[kRoleOut], b.ld[kRoleOut], tl.c0)) &&
+                   (!wp || vec8_ok(wp, b.dtype[kRoleW], b.ld[kRoleW], tl.c0));
+  const int32_t runs = vec ? tl.w / 8 : 0;
+  const int32_t rest = tl.w - 8 * runs;
+  const int32_t rows = i1 - i0;
+  for (int32_t k = threadIdx.x; k < rows * runs; k += blockDim.x) {
+    const int32_t i = i0 + k / runs, j = 8 * (k % runs);
+    float o[8];
+    if (tl.transposed) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = x[static_cast<int64_t>(j + e) * a.m + i];
+    } else {
+      const float4 *xi = reinterpret_cast<const float4 *>(x + static_cast<int64_t>(i) * a.m + j);
+      const float4 p0 = xi[0], p1 = xi[1];
+      o[0] = p0.x; o[1] = p0.y; o[2] = p0.z; o[3] = p0.w;
+      o[4] = p1.x; o[5] = p1.y; o[6] = p1.z; o[7] = p1.w;
+    }
+    if (out) st8_16(out, b.dtype[kRoleOut], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleOut] + tl.c0 + j, o);
+    if (wp) {
+      const int64_t gi = static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleW] + tl.c0 + j;
+      float w[8];
+      ld8_16(wp, b.dtype[kRoleW], gi, w);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = fmaf(-a.lr, o[e], w[e]);
+      st8_16(wp, b.dtype[kRoleW], gi, w);
+    }
+  }
+  for (int32_t k = threadIdx.x; k < rows * rest; k += blockDim.x) {
+    const int32_t i = i0 + k / rest, j = 8 * runs + k % rest;
+    const int64_t xo = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
+    const float o = x[xo];
+    if (out) st_elem(out, b.dtype[kRoleOut], static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleOut] + tl.c0 + j, o);
+    if (wp) {
+      const int64_t gi = static_cast<int64_t>(tl.r0 + i) * b.ld[kRoleW] + tl.c0 + j;
+      st_elem(wp, b.dtype[kRoleW], gi, fmaf(-a.lr, o, ld_elem(wp, b.dtype[kRoleW], gi)));
     }
   }
 }
