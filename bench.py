@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 QUINTIC = (3.4445, -4.7750, 2.0315)
 K_STEPS = 5
+AUTO_CANDIDATES = (128, 256, 512, 0)    # T = 32 / 64 cost more than 128 on chip and couple less
 MU, LR = 0.95, 0.02
 METRIC = "tiled-NS step: matrix elements/s"
 
@@ -233,8 +234,22 @@ def run_ours(args):
     mats, W, M, G = make_state(device, seed_base=1000 * rank, layers=args.layers)
     splits = [s for (_, s) in mats]
     elements = sum(H * Wd for (H, Wd), _ in mats)
-    n_tiles, flops = workload_tiles(mats, T)
-    p = hm.params(T, QUINTIC, steps=K_STEPS, compute=compute)
+    tiles = None
+    if args.budget_ms is not None:
+        # runtime tile-size choice: per matrix, the largest T whose measured
+        # step cost keeps the set within the budget (untimed, before warm-up)
+        from tiled_newton_schulz_b200 import schedule
+        costs = schedule.measure_costs([s for s, _ in mats], splits, candidates=AUTO_CANDIDATES, compute=compute,
+                                       reps=2, device=device, op="step")
+        tiles = schedule.choose_tiles(costs, args.budget_ms / 1e3)
+        modeled_ms = schedule.modeled_cost(costs, tiles) * 1e3
+        n_tiles, flops = 0, 0.0
+        for m, t in zip(mats, tiles):
+            a, b = workload_tiles([m], t if t > 0 else 1 << 30)
+            n_tiles, flops = n_tiles + a, flops + b
+    else:
+        n_tiles, flops = workload_tiles(mats, T)
+    p = hm.params(T, QUINTIC, steps=K_STEPS, compute=compute, tiles=tiles)
     ws_need = hm.workspace_size(M, p, hm.OP_MOMENTUM_STEP, splits)
     ws = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=device) if ws_need else None
     stream = torch.cuda.current_stream(device)
@@ -298,6 +313,8 @@ def run_ours(args):
         per = max(1, -(-n_mat // 16))
         per = -(-per // 5) * 5 if n_mat % 5 == 0 else per     # whole layers (5 matrices each)
         chunks = [list(range(i, min(n_mat, i + per))) for i in range(0, n_mat, per)]
+        p_chunk = [p if tiles is None else hm.params(T, QUINTIC, steps=K_STEPS, compute=compute,
+                                                     tiles=[tiles[i] for i in idx]) for idx in chunks]
         s_in, s_cmp, s_out = (torch.cuda.Stream(device) for _ in range(3))
 
         def e2e_step():
@@ -306,7 +323,7 @@ def run_ours(args):
             for s in (s_in, s_cmp, s_out):
                 s.wait_event(start)
             done_out = None
-            for idx in chunks:
+            for idx, pc in zip(chunks, p_chunk):
                 with torch.cuda.stream(s_in):
                     for i in idx:
                         W[i].copy_(hW[i], non_blocking=True)
@@ -315,7 +332,7 @@ def run_ours(args):
                     e_in = torch.cuda.Event()
                     e_in.record(s_in)
                 s_cmp.wait_event(e_in)
-                hm.momentum_step([W[i] for i in idx], [M[i] for i in idx], [G[i] for i in idx], MU, LR, p,
+                hm.momentum_step([W[i] for i in idx], [M[i] for i in idx], [G[i] for i in idx], MU, LR, pc,
                                  splits=[splits[i] for i in idx], workspace=ws, stream=s_cmp)
                 e_c = torch.cuda.Event()
                 e_c.record(s_cmp)
@@ -348,7 +365,7 @@ def run_ours(args):
 
     # CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 only
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu and tiles is None:
         idx = 1  # layer 0, O projection (4096 x 4096)
         sample = tuple(x[idx][:T].detach().double().cpu().numpy() for x in (W, M, G))
         v, e, dt, threads, desc = cpu_oracle_sample(sample, T, args.cpu_budget)
@@ -359,11 +376,12 @@ def run_ours(args):
     peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     peak_burst = float(peaks.get("bf16_tflops"))
     # the step is a single launch of the on-chip kernel: launch duration = step time
+    # (with per-matrix tile sizes it is several launches; the figure is then the step's)
     achieved = flops / (ms_step / 1e3) / 1e12
-    prof = load_profile_traffic(T)
+    prof = load_profile_traffic(T) if tiles is None else None
     roofline = {
         "bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
-        "traffic": prof, "kernel": "ns_resident_kernel",
+        "traffic": prof, "kernel": "ns_resident_kernel" if tiles is None else "whole step (on-chip and staged launches)",
         "peak_source": f"bf16_tflops_sustained ({peak_src})",
         "frac_of_burst_peak": achieved / peak_burst,
         "flops_per_launch": flops, "flop_count": "nominal: 2(2a+1)n^3 per NS step per tile (a = m/n)",
@@ -375,7 +393,9 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": args.compute, "data": "synthetic",
-        "config": {"workload": f"llama7b_{args.layers}l_full_step_T{T}", "tile": T, "steps_K": K_STEPS, "mu": MU, "lr": LR,
+        "config": {"workload": (f"llama7b_{args.layers}l_full_step_T{T}" if tiles is None else
+                                f"llama7b_{args.layers}l_full_step_autoT_budget{args.budget_ms:g}ms"),
+                   "tile": T if tiles is None else "per matrix", "steps_K": K_STEPS, "mu": MU, "lr": LR,
                    "matrices": len(mats), "split_blocks": sum(len(s[1]) if s else 1 for s in splits),
                    "tiles": n_tiles, "elements_per_gpu": elements, "storage": "bf16 W, M, G",
                    "accumulate": "fp32",
@@ -388,6 +408,13 @@ def run_ours(args):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if tiles is not None:
+        mix = {}
+        for t in tiles:
+            mix[str(t if t > 0 else "whole")] = mix.get(str(t if t > 0 else "whole"), 0) + 1
+        line["config"].update({"tile_mix": mix, "candidates": list(AUTO_CANDIDATES), "budget_ms": args.budget_ms,
+                               "modeled_ms": modeled_ms,
+                               "cost_model": "momentum_step per matrix at each T, CUDA events, batched per shape"})
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -425,6 +452,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--budget-ms", type=float, default=None,
+                    help="choose T per matrix at run time: the largest tiles whose measured cost fits this budget")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

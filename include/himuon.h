@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define HIMUON_VERSION 1
+#define HIMUON_VERSION 2   /* 2: himuon_ns_params.tiles */
 
 #if defined(__GNUC__)
 #define HIMUON_API __attribute__((visibility("default")))
@@ -112,7 +112,23 @@ typedef struct {
                               (X <- Q X, R <- X X^T, Q <- I); the page restarts at t = 3         */
   int64_t chunk_bytes;     /* staged path: upper bound on the scratch one chunk of tiles may
                               use (memory-bounded chunking); 0 = use all of ws_bytes             */
+  const int32_t *tiles;    /* host, NULL or one T per matrix (a runtime tile-size schedule,
+                              "Hierarchical Muon" abstract): tiles[i] replaces `tile` for matrix
+                              i (and all its split blocks), with the same meaning (<= 0: the
+                              whole matrix).  See "Per-matrix tile sizes" below.                 */
 } himuon_ns_params;
+
+/*
+ * Per-matrix tile sizes (p->tiles != NULL).  The matrices of a call are
+ * grouped by their T (in first-appearance order of T, matrix order kept inside
+ * a group), and each group runs as the same call would with p->tile = that T:
+ * on chip for T <= 128, staged otherwise.  The groups run one after another on
+ * `stream` and share `ws`, which must hold the largest group's need (what
+ * himuon_workspace_size returns for the same params).  Every group's arguments
+ * are checked before the first is enqueued.  himuon_ns_full ignores `tiles`
+ * (every matrix is one tile); himuon_ns_static rejects it with
+ * HIMUON_ERR_UNSUPPORTED.
+ */
 
 /* op codes for himuon_workspace_size */
 enum { HIMUON_OP_NS_TILED = 0, HIMUON_OP_NS_FULL = 1, HIMUON_OP_GRAM_NS = 2, HIMUON_OP_MOMENTUM_STEP = 3 };

@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.himuon_version() == 1
+    assert lib.himuon_version() == 2
     assert himuon.status_string(0) == "ok"
     assert "workspace" in himuon.status_string(-3)
 
@@ -95,3 +95,28 @@ def test_workspace_size_on_the_host(lib):
     assert need > 256 * 256 * 8 * 256
     pc = himuon.params(256, (3.4445, -4.7750, 2.0315), steps=5, chunk_bytes=64 << 20)
     assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(pc), 0) <= 64 << 20
+
+
+def test_per_matrix_tiles_on_the_host(lib):
+    """p->tiles: the workspace is the largest group's need; the fixed-scratch
+    entry point rejects it; a bad matrix in any group fails the whole call."""
+    Q = (3.4445, -4.7750, 2.0315)
+    shapes = [(4096, 4096), (1024, 4096), (2048, 2048)]
+    mats = (himuon.Mat * 3)(*[himuon.Mat(0x1000 * (i + 1), r, c, c, himuon.BF16) for i, (r, c) in enumerate(shapes)])
+    one = lambda i: (himuon.Mat * 1)(mats[i])
+    per = []
+    for i, T in enumerate((128, 256, 0)):
+        per.append(lib.himuon_workspace_size(one(i), 1, None, ctypes.byref(himuon.params(T, Q, steps=5)),
+                                             himuon.OP_NS_TILED if T > 0 else himuon.OP_NS_FULL))
+    assert per[0] == 0 and per[1] > 0 and per[2] > 0
+    pt = himuon.params(128, Q, steps=5, tiles=[128, 256, 0])
+    for op in (himuon.OP_NS_TILED, himuon.OP_MOMENTUM_STEP):
+        assert lib.himuon_workspace_size(mats, 3, None, ctypes.byref(pt), op) == max(per)
+    # all on chip -> no workspace; ns_full ignores tiles
+    assert lib.himuon_workspace_size(mats, 3, None, ctypes.byref(himuon.params(0, Q, steps=5, tiles=[128] * 3)),
+                                     himuon.OP_NS_TILED) == 0
+    full = lib.himuon_workspace_size(mats, 3, None, ctypes.byref(himuon.params(0, Q, steps=5)), himuon.OP_NS_FULL)
+    assert lib.himuon_workspace_size(mats, 3, None, ctypes.byref(pt), himuon.OP_NS_FULL) == full
+    assert lib.himuon_ns_static(mats, mats, 3, None, ctypes.byref(pt), None) == -2
+    bad = (himuon.Mat * 3)(mats[0], mats[1], himuon.Mat(0, 2048, 2048, 2048, himuon.BF16))
+    assert lib.himuon_ns_tiled(bad, bad, 3, None, ctypes.byref(pt), None, 0, None) == -1

@@ -290,7 +290,7 @@ struct PlanCache {
   std::mutex mu;   // lookups from several host threads do not corrupt the cache
   std::list<std::pair<std::string, std::shared_ptr<Plan>>> lru;
   std::map<std::string, std::list<std::pair<std::string, std::shared_ptr<Plan>>>::iterator> index;
-  static constexpr size_t kCap = 32;
+  static constexpr size_t kCap = 64;   // a per-matrix-T call takes one entry per tile size
 };
 PlanCache &cache() {
   static PlanCache *c = new PlanCache();  // never destroyed: avoids freeing at exit after the context is gone
@@ -750,27 +750,147 @@ int run_resident(const Plan &plan, int op, const himuon_ns_params &p, float mu, 
   return launch_ns_resident(a, grid, stream) == cudaSuccess ? HIMUON_OK : HIMUON_ERR_CUDA;
 }
 
-int dispatch(int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params *p, float mu, float lr,
-             void *ws, size_t ws_bytes, void *stream) {
+// One call's checks and plan, kept apart from its launch so that a call with
+// per-matrix tile sizes can check every group before enqueuing the first.
+struct Prepared {
+  int op = 0;
+  std::shared_ptr<Plan> plan;
+  himuon_ns_params p{};
+  bool has_w = false, has_o = false;
+};
+
+int prepare(int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params *p, void *ws,
+            size_t ws_bytes, Prepared &pr) {
   int rc = check_params(p);
   if (rc) return rc;
   rc = check_call(cm, splits);
   if (rc) return rc;
   rc = check_device();
   if (rc) return rc;
-  std::shared_ptr<Plan> plan;
-  rc = get_plan(op, cm, splits, *p, plan);
+  rc = get_plan(op, cm, splits, *p, pr.plan);
   if (rc) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (plan->path == kPathResident) {
-    const bool has_w = op == HIMUON_OP_MOMENTUM_STEP && cm.role[kRoleW];
-    const bool has_o = cm.role[kRoleOut] != nullptr;
-    return run_resident(*plan, op, *p, mu, lr, has_w, has_o, s);
-  }
-  const int64_t need = staged_ws_bytes(*plan, p->compute, op == HIMUON_OP_GRAM_NS);
+  pr.op = op;
+  pr.p = *p;
+  pr.has_w = op == HIMUON_OP_MOMENTUM_STEP && cm.role[kRoleW];
+  pr.has_o = cm.role[kRoleOut] != nullptr;
+  if (pr.plan->path == kPathResident) return HIMUON_OK;
+  const int64_t need = staged_ws_bytes(*pr.plan, p->compute, op == HIMUON_OP_GRAM_NS);
   if (!ws || static_cast<int64_t>(ws_bytes) < need) return HIMUON_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return HIMUON_ERR_ALIGNMENT;
-  return run_staged(*plan, op, *p, mu, lr, ws, ws_bytes, s);
+  return HIMUON_OK;
+}
+
+int launch(const Prepared &pr, float mu, float lr, void *ws, size_t ws_bytes, void *stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pr.plan->path == kPathResident) return run_resident(*pr.plan, pr.op, pr.p, mu, lr, pr.has_w, pr.has_o, s);
+  return run_staged(*pr.plan, pr.op, pr.p, mu, lr, ws, ws_bytes, s);
+}
+
+// Matrices of a call regrouped by their tile size (p->tiles): per group, the
+// role arrays and splits of its matrices in call order, and the params with
+// `tile` set to the group's T.
+struct TileGroup {
+  int32_t T = 0;
+  std::vector<int32_t> idx;
+  std::vector<himuon_mat> role[kNumRoles];
+  std::vector<himuon_split> splits;
+  CallMats cm;
+  himuon_ns_params p{};
+};
+
+int group_by_tile(const CallMats &cm, const himuon_split *splits, const himuon_ns_params *p,
+                  std::vector<TileGroup> &groups) {
+  if (cm.n < 1) return HIMUON_ERR_INVALID;
+  groups.clear();
+  for (int32_t i = 0; i < cm.n; ++i) {
+    const int32_t T = p->tiles[i] <= 0 ? 0 : p->tiles[i];
+    size_t g = 0;
+    while (g < groups.size() && groups[g].T != T) ++g;
+    if (g == groups.size()) {
+      groups.emplace_back();
+      groups.back().T = T;
+    }
+    groups[g].idx.push_back(i);
+  }
+  for (TileGroup &g : groups) {
+    g.cm.n = static_cast<int32_t>(g.idx.size());
+    for (int r = 0; r < kNumRoles; ++r) {
+      if (!cm.role[r]) continue;
+      for (int32_t i : g.idx) g.role[r].push_back(cm.role[r][i]);
+      g.cm.role[r] = g.role[r].data();
+    }
+    if (splits)
+      for (int32_t i : g.idx) g.splits.push_back(splits[i]);
+    g.p = *p;
+    g.p.tile = g.T;
+    g.p.tiles = nullptr;
+  }
+  return HIMUON_OK;
+}
+
+// Tiled NS picks full-matrix NS for T <= 0; the other ops take T as given.
+int group_op(int op, int32_t T) {
+  if (op == HIMUON_OP_NS_TILED || op == HIMUON_OP_NS_FULL) return T <= 0 ? HIMUON_OP_NS_FULL : HIMUON_OP_NS_TILED;
+  return op;
+}
+
+int dispatch(int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params *p, float mu, float lr,
+             void *ws, size_t ws_bytes, void *stream) {
+  if (p && p->tiles) {
+    int rc = check_params(p);   // the whole call first: same error precedence as one group
+    if (rc) return rc;
+    rc = check_call(cm, splits);
+    if (rc) return rc;
+    std::vector<TileGroup> groups;
+    rc = group_by_tile(cm, splits, p, groups);
+    if (rc) return rc;
+    std::vector<Prepared> prep(groups.size());
+    for (size_t g = 0; g < groups.size(); ++g) {
+      rc = prepare(group_op(op, groups[g].T), groups[g].cm, splits ? groups[g].splits.data() : nullptr, &groups[g].p,
+                   ws, ws_bytes, prep[g]);
+      if (rc) return rc;
+    }
+    for (const Prepared &pr : prep) {
+      rc = launch(pr, mu, lr, ws, ws_bytes, stream);
+      if (rc) return rc;
+    }
+    return HIMUON_OK;
+  }
+  Prepared pr;
+  const int rc = prepare(op, cm, splits, p, ws, ws_bytes, pr);
+  if (rc) return rc;
+  return launch(pr, mu, lr, ws, ws_bytes, stream);
+}
+
+// Device scratch of one call with a single tile size (arguments checked).
+int64_t workspace_one(const CallMats &cm, const himuon_split *splits, const himuon_ns_params &p, int op) {
+  std::vector<HostBlock> blocks;
+  int64_t n_tiles = 0;
+  const int64_t tile = op == HIMUON_OP_NS_FULL ? 0 : p.tile;
+  int rc = make_blocks(cm, splits, tile, blocks, &n_tiles);
+  if (rc) return rc;
+  if (op != HIMUON_OP_GRAM_NS && !force_staged() && resident_pack(cm, blocks, p) > 0) return 0;
+  // staged: one tile of the largest class is the minimum; a full chunk of every
+  // class makes the call run in one chunk per class.
+  int64_t need = 0;
+  std::map<std::pair<int64_t, int64_t>, int64_t> counts;
+  for (const HostBlock &b : blocks)
+    for (int64_t tr = 0; tr < b.tiles_r; ++tr)
+      for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
+        const int64_t h = std::min(b.T, b.rows - tr * b.T), w = std::min(b.T, b.cols - tc * b.T);
+        counts[{round_up(std::min(h, w), 128), round_up(std::max(h, w), 128)}] += 1;
+      }
+  for (auto &kv : counts) {
+    int64_t k = std::min<int64_t>(kv.second, 65535);
+    int64_t bytes = static_cast<int64_t>(ws_layout(kv.first.first, kv.first.second, k, p.compute,
+                                                   op == HIMUON_OP_GRAM_NS).total);
+    if (p.chunk_bytes > 0 && bytes > p.chunk_bytes)
+      bytes = std::max<int64_t>(p.chunk_bytes, static_cast<int64_t>(ws_layout(kv.first.first, kv.first.second, 1,
+                                                                                p.compute, op == HIMUON_OP_GRAM_NS)
+                                                                          .total));
+    need = std::max(need, bytes);
+  }
+  return need;
 }
 
 }  // namespace
@@ -882,7 +1002,8 @@ int himuon_ns_tiled(const himuon_mat *in, const himuon_mat *out, int32_t n, cons
   cm.n = n;
   cm.role[kRoleIn] = in;
   cm.role[kRoleOut] = out;
-  const int op = (p->tile <= 0) ? HIMUON_OP_NS_FULL : HIMUON_OP_NS_TILED;
+  // with per-matrix tile sizes each group picks tiled or full NS by its own T
+  const int op = (p->tiles || p->tile > 0) ? HIMUON_OP_NS_TILED : HIMUON_OP_NS_FULL;
   return dispatch(op, cm, splits, p, 0.f, 0.f, ws, ws_bytes, stream);
 }
 
@@ -893,7 +1014,9 @@ int himuon_ns_full(const himuon_mat *in, const himuon_mat *out, int32_t n, const
   cm.n = n;
   cm.role[kRoleIn] = in;
   cm.role[kRoleOut] = out;
-  return dispatch(HIMUON_OP_NS_FULL, cm, splits, p, 0.f, 0.f, ws, ws_bytes, stream);
+  himuon_ns_params q = *p;   // every matrix is one tile: a per-matrix T does not apply
+  q.tiles = nullptr;
+  return dispatch(HIMUON_OP_NS_FULL, cm, splits, &q, 0.f, 0.f, ws, ws_bytes, stream);
 }
 
 int himuon_gram_ns(const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,
@@ -932,31 +1055,15 @@ int64_t himuon_workspace_size(const himuon_mat *mats, int32_t n, const himuon_sp
   if (op == HIMUON_OP_MOMENTUM_STEP) cm.role[kRoleOut] = nullptr;
   rc = check_call(cm, splits);
   if (rc) return rc;
-  std::vector<HostBlock> blocks;
-  int64_t n_tiles = 0;
-  const int64_t tile = op == HIMUON_OP_NS_FULL ? 0 : p->tile;
-  rc = make_blocks(cm, splits, tile, blocks, &n_tiles);
+  if (!p->tiles || op == HIMUON_OP_NS_FULL) return workspace_one(cm, splits, *p, op);
+  std::vector<TileGroup> groups;
+  rc = group_by_tile(cm, splits, p, groups);
   if (rc) return rc;
-  if (op != HIMUON_OP_GRAM_NS && !force_staged() && resident_pack(cm, blocks, *p) > 0) return 0;
-  // staged: one tile of the largest class is the minimum; a full chunk of every
-  // class makes the call run in one chunk per class.
   int64_t need = 0;
-  std::map<std::pair<int64_t, int64_t>, int64_t> counts;
-  for (const HostBlock &b : blocks)
-    for (int64_t tr = 0; tr < b.tiles_r; ++tr)
-      for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
-        const int64_t h = std::min(b.T, b.rows - tr * b.T), w = std::min(b.T, b.cols - tc * b.T);
-        counts[{round_up(std::min(h, w), 128), round_up(std::max(h, w), 128)}] += 1;
-      }
-  for (auto &kv : counts) {
-    int64_t k = std::min<int64_t>(kv.second, 65535);
-    int64_t bytes = static_cast<int64_t>(ws_layout(kv.first.first, kv.first.second, k, p->compute,
-                                                   op == HIMUON_OP_GRAM_NS).total);
-    if (p->chunk_bytes > 0 && bytes > p->chunk_bytes)
-      bytes = std::max<int64_t>(p->chunk_bytes, static_cast<int64_t>(ws_layout(kv.first.first, kv.first.second, 1,
-                                                                                p->compute, op == HIMUON_OP_GRAM_NS)
-                                                                          .total));
-    need = std::max(need, bytes);
+  for (const TileGroup &g : groups) {
+    const int64_t b = workspace_one(g.cm, splits ? g.splits.data() : nullptr, g.p, group_op(op, g.T));
+    if (b < 0) return b;
+    need = std::max(need, b);
   }
   return need;
 }

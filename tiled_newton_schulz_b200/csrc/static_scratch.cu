@@ -50,6 +50,7 @@ int scratch_address(void **out) {
 extern "C" int himuon_ns_static(const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,
                                 const himuon_ns_params *p, void *stream) {
   if (!in || !out || !p) return HIMUON_ERR_INVALID;
+  if (p->tiles) return HIMUON_ERR_UNSUPPORTED;   // one tile size per call here
   void *scratch = nullptr;
   const int rc = himuon::scratch_address(&scratch);
   if (rc != HIMUON_OK) return rc;

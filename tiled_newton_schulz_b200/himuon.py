@@ -38,7 +38,7 @@ class Params(ctypes.Structure):
     _fields_ = [("tile", ctypes.c_int32), ("steps", ctypes.c_int32), ("coeffs", ctypes.POINTER(ctypes.c_float)),
                 ("eps", ctypes.c_float), ("compute", ctypes.c_int32), ("safety", ctypes.c_float),
                 ("n_restart", ctypes.c_int32), ("restart_at", ctypes.POINTER(ctypes.c_int32)),
-                ("chunk_bytes", ctypes.c_int64)]
+                ("chunk_bytes", ctypes.c_int64), ("tiles", ctypes.POINTER(ctypes.c_int32))]
 
 
 class HimuonError(RuntimeError):
@@ -129,7 +129,11 @@ def _splits(splits, n):
 
 
 def params(tile: int, coeffs, steps: int | None = None, eps: float = 1e-7, compute: int = BF16,
-           safety: float = 1.0, restart: Sequence[int] = (), chunk_bytes: int = 0):
+           safety: float = 1.0, restart: Sequence[int] = (), chunk_bytes: int = 0,
+           tiles: Sequence[int] | None = None):
+    """himuon_ns_params.  `tiles`: None, or one T per matrix of the call (it
+    then replaces `tile`; T <= 0 is the whole matrix), e.g. the output of a
+    runtime tile-size schedule (``schedule.TileSchedule``, ``schedule.choose_tiles``)."""
     flat = [float(v) for tri in (coeffs if isinstance(coeffs[0], (list, tuple)) else [coeffs]) for v in tri]
     if steps is not None and len(flat) == 3:
         flat = flat * steps
@@ -137,8 +141,12 @@ def params(tile: int, coeffs, steps: int | None = None, eps: float = 1e-7, compu
     c = (ctypes.c_float * len(flat))(*flat)
     r = (ctypes.c_int32 * max(1, len(restart)))(*restart)
     p = Params(int(tile), K, ctypes.cast(c, ctypes.POINTER(ctypes.c_float)), float(eps), int(compute), float(safety),
-               len(restart), ctypes.cast(r, ctypes.POINTER(ctypes.c_int32)), int(chunk_bytes))
-    p._keep = (c, r)
+               len(restart), ctypes.cast(r, ctypes.POINTER(ctypes.c_int32)), int(chunk_bytes), None)
+    tl = None
+    if tiles is not None:
+        tl = (ctypes.c_int32 * max(1, len(tiles)))(*[int(t) for t in tiles])
+        p.tiles = ctypes.cast(tl, ctypes.POINTER(ctypes.c_int32))
+    p._keep = (c, r, tl)
     return p
 
 
@@ -179,8 +187,12 @@ def _ns_call(fn_name, op, inputs, outputs, p, splits, workspace, stream):
     return _ws
 
 
+def _has_tiles(p: Params) -> bool:
+    return bool(ctypes.cast(p.tiles, ctypes.c_void_p).value)
+
+
 def ns_tiled(inputs, outputs, p: Params, splits=None, workspace=None, stream=None):
-    op = OP_NS_FULL if p.tile <= 0 else OP_NS_TILED
+    op = OP_NS_TILED if (_has_tiles(p) or p.tile > 0) else OP_NS_FULL
     return _ns_call("himuon_ns_tiled", op, inputs, outputs, p, splits, workspace, stream)
 
 
