@@ -327,6 +327,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     while (ti * (ti + 1) / 2 > k) --ti;
     m0 = ti * 128;
     n0 = (k - ti * (ti + 1) / 2) * 128;
+  } else if (gridDim.y > 1) {
+    // Grouped order: the CTAs launched together cover bands of up to 32 row
+    // tiles, row tile fastest, so one wave shares each B column panel among
+    // the band's rows and keeps the band's A row panels in L2 while B streams
+    // through once (row-major order re-read all of B for every ~2 row tiles).
+    const int64_t gx = gridDim.x, gy = gridDim.y;
+    const int64_t L = static_cast<int64_t>(blockIdx.y) * gx + blockIdx.x;   // launch order
+    const int64_t G = gy < 32 ? gy : 32;
+    const int64_t per = G * gx, g = L / per, r = L % per;
+    const int64_t gm = (gy - g * G) < G ? (gy - g * G) : G;
+    m0 = static_cast<int32_t>((g * G + r % gm) * 128);
+    n0 = static_cast<int32_t>((r / gm) * 128);
   }
   const bool mirror = a.ep.sym && m0 != n0;
   const int nk = static_cast<int>(a.K / 64);
