@@ -268,7 +268,7 @@ def test_integer_coded_reassembly_bitexact(hm, T):
     assert np.array_equal(np.sign(y), np.sign(xin))
 
 
-@pytest.mark.parametrize("restart", [(3,), ()])
+@pytest.mark.parametrize("restart", [(3,), (), (2, 4), (2, 3), (1,)])
 def test_gram_ns_fp16(hm, restart):
     n, m = 256, 1024
     X = inputs.low_rank_plus_noise(n, m, inputs.sigma_exp(n, 32.0), 1e-3, seed=4)
@@ -281,6 +281,19 @@ def test_gram_ns_fp16(hm, restart):
     yy = to_np(y)
     assert np.linalg.norm(yy - ref) / np.linalg.norm(ref) <= TOL16
     assert max_sv_diff(yy, ref, 0) <= SVTOL
+
+
+@pytest.mark.parametrize("restart", [(3,), (2, 4)])
+def test_gram_ns_fp32(hm, restart):
+    """Gram NS with fp32 storage and arithmetic (CUDA-core products) against
+    the oracle within the fp32 tolerance; restarts before steps 3, or 2 and 4."""
+    X = inputs.gaussian((256, 1024), seed=41)
+    x = dev(X, torch.float32)
+    y = torch.empty_like(x)
+    hm.gram_ns([x], [y], hm.params(0, QUINTIC, steps=5, compute=hm.FP32, restart=restart))
+    assert hm.device_status() == 0
+    ref = oracle.gram_ns(to_np(x), C32, restart=restart)
+    assert np.linalg.norm(to_np(y) - ref) / np.linalg.norm(ref) <= TOL32
 
 
 @pytest.mark.parametrize("T", [128, 256])

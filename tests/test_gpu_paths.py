@@ -97,3 +97,37 @@ def test_resume_from_saved_state_is_bit_identical(hm):
     hm.momentum_step([w_r], [m_r], [g2], 0.95, 0.02, p)
     assert hm.device_status() == 0
     assert torch.equal(w, w_r) and torch.equal(m, m_r)
+
+
+def partial_signed_permutation(H, W, k, seed):
+    """H x W (H <= W) with one +-1 per row, in column (k i + 5) mod W: distinct
+    columns when gcd(k, W) = 1, so X X^T = I and every singular value is 1."""
+    assert np.gcd(k, W) == 1 and H <= W
+    P = np.zeros((H, W))
+    P[np.arange(H), (np.arange(H) * k + 5) % W] = np.random.default_rng(seed).choice([-1.0, 1.0], H)
+    return P
+
+
+@pytest.mark.parametrize("H,W", [(4608, 4608), (4224, 8320)])
+def test_full_ns_of_permutation_beyond_one_band_of_row_tiles(hm, H, W):
+    """Full NS where the staged GEMMs have more than 32 row tiles (36 and 33:
+    a full band of 32 and a partial one in the grouped CTA order).  X is a
+    signed (partial) permutation, so every product is exact up to the operand
+    rounding and NS(X) = phi(1/sqrt(H)) X: the output's support and signs must
+    equal X's exactly, every magnitude must be the same, and that magnitude is
+    the oracle's map of a 2 x 2 matrix with the same normalised singular value
+    (diag(1, sqrt(H - 1)) has Frobenius norm sqrt(H)).  A GEMM tile written to
+    the wrong place, or not written, breaks the support."""
+    X = partial_signed_permutation(H, W, 7, seed=H)
+    x = dev(X)
+    y = torch.empty_like(x)
+    hm.ns_full([x], [y], hm.params(0, QUINTIC, steps=5))
+    assert hm.device_status() == 0
+    Y = to_np(y)
+    nz = X != 0
+    assert np.array_equal(Y != 0, nz)
+    assert np.array_equal(np.sign(Y[nz]), np.sign(X[nz]))
+    mags = np.abs(Y[nz])
+    assert np.all(mags == mags[0])
+    want = oracle.ns_map(np.diag([1.0, np.sqrt(H - 1.0)]), C32)[0, 0]
+    assert abs(mags[0] - want) <= TOL16 * want

@@ -645,11 +645,19 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
         auto rzop = [&]() -> void * { return f32 ? static_cast<void *>(rz32) : rz16; };
         auto qop = [&](int i) -> void * { return f32 ? static_cast<void *>(qf[i]) : q16[i]; };
         bool q_identity = true;
+        auto restarts_at = [&p](int t) {
+          for (int i = 0; i < p.n_restart; ++i)
+            if (p.restart_at[i] == t) return true;
+          return false;
+        };
         rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, sym(epi(1.f, 0.f, nullptr, r32, r16, dt16)));
         for (int t = 1; t <= p.steps && rc == HIMUON_OK; ++t) {
           const float a = p.coeffs[3 * (t - 1)], b = p.coeffs[3 * (t - 1) + 1], cc = p.coeffs[3 * (t - 1) + 2];
-          bool restart = false;
-          for (int i = 0; i < p.n_restart; ++i) restart |= p.restart_at[i] == t;
+          const bool restart = restarts_at(t);
+          // After the last step, or before a restart (which rebuilds R from the
+          // new X and resets Q), this step's R, RZ and fp32 Q are never read:
+          // those products and writes are skipped (the results are unchanged).
+          const bool last_use = t == p.steps || restarts_at(t + 1);
           if (restart) {
             if (!q_identity) {  // X <- Q X
               if (f32) {
@@ -666,8 +674,10 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
             }
             q_identity = true;
           }
-          // Z = b R + c R^2
-          rc = ops.mm(rop(), n, n, rop(), n, n, 0, n, n, n, bc, sym(epi(cc, b, r32, z32, z16, dt16)));
+          // Z = b R + c R^2 (its fp32 copy feeds only Q = Z + aI right after Q = I,
+          // or every product when the operands are fp32)
+          rc = ops.mm(rop(), n, n, rop(), n, n, 0, n, n, n, bc,
+                      sym(epi(cc, b, r32, (f32 || q_identity) ? z32 : nullptr, z16, dt16)));
           if (rc) break;
           // Q <- Q Z + a Q
           if (q_identity) {
@@ -675,11 +685,12 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
             q_identity = false;
           } else {
             rc = ops.mm(qop(qc), n, n, zop(), n, n, 0, n, n, n, bc,
-                        sym(epi(1.f, a, qf[qc], qf[1 - qc], f32 ? nullptr : q16[1 - qc], dt16)));
+                        sym(epi(1.f, a, qf[qc], (f32 || !last_use) ? qf[1 - qc] : nullptr,
+                                f32 ? nullptr : q16[1 - qc], dt16)));
             qc = 1 - qc;
             if (rc) break;
           }
-          if (t == p.steps) break;   // R_K is never used
+          if (last_use) continue;   // R_K, and R before a restart, are never used
           // RZ <- R Z + a R
           rc = ops.mm(rop(), n, n, zop(), n, n, 0, n, n, n, bc, sym(epi(1.f, a, r32, rz32, rz16, dt16)));
           if (rc) break;
