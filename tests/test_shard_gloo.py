@@ -1,12 +1,16 @@
 """Multi-rank path on CPU (gloo, world_size 2): matrices are assigned to ranks
 by FLOPs, each rank runs the fp64 oracle on its own matrices, the results are
 gathered, and rank 0 checks they equal the single-process result bit for bit
-and that every matrix was processed exactly once."""
+and that every matrix was processed exactly once.  The sharded Muon step
+(gradients reduced onto owners, the owner's step, weights broadcast) runs with
+the oracle as its step function and must equal the single-process step on the
+averaged gradients; incomplete inputs on one rank make every rank raise."""
 import os
 import socket
 
 import numpy as np
 import pytest
+import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
@@ -76,3 +80,94 @@ def test_assignment_covers_each_matrix_once_and_balances():
         flat = sorted(i for lst in a for i in lst)
         assert flat == list(range(len(shapes)))
         assert shard.imbalance(shapes, splits, 128, a) < 1.05
+
+
+MU, LR = 0.95, 0.02
+
+
+def _oracle_step(T):
+    """Step function with the library's signature, computed by the fp64 oracle
+    in place on CPU tensors (the sharded step calls the library on a GPU)."""
+    import oracle
+
+    def step(W, M, G, mu, lr, p, splits=None):
+        for k in range(len(W)):
+            sp = None if splits is None else splits[k]
+            mp = oracle.momentum(M[k].numpy(), G[k].numpy(), mu)
+            O = oracle.ns_tiled_split(mp, T, [inputs.QUINTIC] * 5, split=sp)
+            M[k].copy_(torch.from_numpy(mp))
+            W[k].sub_(lr * torch.from_numpy(O))
+    return step
+
+
+def _state(rank):
+    W = [torch.from_numpy(0.02 * inputs.gaussian(s, seed=200 + i)) for i, s in enumerate(SHAPES)]
+    M = [torch.from_numpy(inputs.gaussian(s, seed=300 + i)) for i, s in enumerate(SHAPES)]
+    G = [torch.from_numpy(inputs.gaussian(s, seed=400 + 10 * i + rank)) for i, s in enumerate(SHAPES)]
+    return W, M, G
+
+
+def _step_worker(rank, world, port, q, broken):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        assignment = shard.assign_matrices(SHAPES, SPLITS, T, world)
+        W, M, G = _state(rank)
+        own = shard.owners(assignment, len(SHAPES))
+        M = [m if own[i] == rank else None for i, m in enumerate(M)]
+        if broken and rank == 1:
+            M[assignment[1][0]] = None
+        try:
+            shard.sharded_momentum_step(W, M, G, MU, LR, None, assignment, splits=SPLITS, step_fn=_oracle_step(T))
+        except ValueError as e:
+            q.put((rank, "raised", str(e)))
+            return
+        q.put((rank, "done", [w.numpy() for w in W], {i: M[i].numpy() for i in assignment[rank]}))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run_step(broken):
+    import oracle
+    oracle.build()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_step_worker, args=(r, 2, port, q, broken)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(p.exitcode == 0 for p in procs)
+    return sorted(out, key=lambda r: r[0])
+
+
+def test_two_rank_sharded_momentum_step_matches_single_process():
+    import oracle
+    out = _run_step(broken=False)
+    assert [o[1] for o in out] == ["done", "done"]
+    W, M, _ = _state(0)
+    G = [(a + b) / 2 for a, b in zip(_state(0)[2], _state(1)[2])]
+    for i in range(len(SHAPES)):
+        mp = oracle.momentum(M[i].numpy(), G[i].numpy(), MU)
+        Wr = W[i].numpy() - LR * oracle.ns_tiled_split(mp, T, [inputs.QUINTIC] * 5, split=SPLITS[i])
+        for o in out:                       # every rank holds the same new weights
+            assert np.array_equal(o[2][i], Wr), i
+        owner = [o for o in out if i in o[3]]
+        assert len(owner) == 1 and np.array_equal(owner[0][3][i], mp), i
+
+
+def test_sharded_step_with_incomplete_inputs_raises_on_every_rank():
+    out = _run_step(broken=True)
+    assert [o[1] for o in out] == ["raised", "raised"]
+    assert "rank 1 owns a matrix without momentum" in out[1][2]
+    assert "another rank" in out[0][2]
+
+
+def test_owners_rejects_bad_assignments():
+    assert shard.owners([[0, 2], [1]], 3) == [0, 1, 0]
+    with pytest.raises(ValueError):
+        shard.owners([[0, 1], [1]], 3)
+    with pytest.raises(ValueError):
+        shard.owners([[0], [2]], 3)
