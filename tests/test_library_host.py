@@ -120,3 +120,16 @@ def test_per_matrix_tiles_on_the_host(lib):
     assert lib.himuon_ns_static(mats, mats, 3, None, ctypes.byref(pt), None) == -2
     bad = (himuon.Mat * 3)(mats[0], mats[1], himuon.Mat(0, 2048, 2048, 2048, himuon.BF16))
     assert lib.himuon_ns_tiled(bad, bad, 3, None, ctypes.byref(pt), None, 0, None) == -1
+
+
+def test_binding_checks_the_tile_list_length(lib):
+    """The C side reads one T per matrix from params.tiles; the binding
+    refuses a list of another length before calling it."""
+    import torch
+    Q = (3.4445, -4.7750, 2.0315)
+    x = [torch.zeros(16, 16, dtype=torch.bfloat16) for _ in range(3)]
+    with pytest.raises(ValueError):
+        himuon.workspace_size(x, himuon.params(128, Q, steps=5, tiles=[128, 256]), himuon.OP_NS_TILED)
+    with pytest.raises(ValueError):
+        himuon.ns_tiled(x, x, himuon.params(128, Q, steps=5, tiles=[128] * 4))
+    assert himuon.workspace_size(x, himuon.params(128, Q, steps=5, tiles=[128, 0, 256]), himuon.OP_NS_TILED) >= 0

@@ -18,6 +18,8 @@ def test_schedule_milestones_and_overrides():
     assert s.tiles(10, 4) == [64, 64, 0, 64]
     assert s.tiles(999, 4) == [64, 64, 0, 32]
     assert s.tiles(1000, 5) == [256, 256, 0, 32, 256]
+    import numpy as np
+    assert TileSchedule(per_matrix={0: np.int64(256)}).tiles(0, 2) == [256, 128]
     with pytest.raises(ValueError):
         TileSchedule(milestones=[(5, 64), (5, 128)])
     with pytest.raises(ValueError):

@@ -147,7 +147,15 @@ def params(tile: int, coeffs, steps: int | None = None, eps: float = 1e-7, compu
         tl = (ctypes.c_int32 * max(1, len(tiles)))(*[int(t) for t in tiles])
         p.tiles = ctypes.cast(tl, ctypes.POINTER(ctypes.c_int32))
     p._keep = (c, r, tl)
+    p._ntiles = None if tiles is None else len(tiles)
     return p
+
+
+def _check_tiles(p: Params, n: int) -> None:
+    """The library reads one tile size per matrix from p.tiles: the list must
+    have exactly n entries (the C side cannot see its length)."""
+    if _has_tiles(p) and getattr(p, "_ntiles", None) != n:
+        raise ValueError(f"params.tiles has {getattr(p, '_ntiles', '?')} entries for {n} matrices")
 
 
 def _stream(stream):
@@ -157,6 +165,7 @@ def _stream(stream):
 
 
 def workspace_size(tensors, p: Params, op: int, splits=None) -> int:
+    _check_tiles(p, len(tensors))
     m = _mats(tensors)
     sp, _keep = _splits(splits, len(tensors))
     n = load().himuon_workspace_size(m, len(tensors), sp, ctypes.byref(p), op)
@@ -179,6 +188,7 @@ def _workspace(tensors, p, op, splits, workspace):
 def _ns_call(fn_name, op, inputs, outputs, p, splits, workspace, stream):
     if len(inputs) != len(outputs):
         raise ValueError("inputs and outputs differ in length")
+    _check_tiles(p, len(inputs))
     mi, mo = _mats(inputs), _mats(outputs)
     sp, _keep = _splits(splits, len(inputs))
     wp, wb, _ws = _workspace(inputs, p, op, splits, workspace)
@@ -222,6 +232,7 @@ def momentum_step(W, M, G, mu: float, lr: float, p: Params, splits=None, update_
                   stream=None):
     """M <- mu M + G; O = tiledNS(M); W <- W - lr O (W may be None); O to update_out."""
     n = len(M)
+    _check_tiles(p, n)
     mw = _mats(W) if W is not None else None
     mm, mg = _mats(M), _mats(G)
     mo = _mats(update_out) if update_out is not None else None

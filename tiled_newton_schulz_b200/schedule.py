@@ -21,6 +21,7 @@ needs, and the library runs their result in one call
 from __future__ import annotations
 
 import math
+import numbers
 from typing import Mapping, Sequence
 
 
@@ -47,7 +48,7 @@ class TileSchedule:
         self.milestones = self._check(milestones)
         self.per_matrix = {}
         for i, v in (per_matrix or {}).items():
-            self.per_matrix[int(i)] = int(v) if isinstance(v, (int,)) else self._check(v)
+            self.per_matrix[int(i)] = int(v) if isinstance(v, numbers.Integral) else self._check(v)
 
     @staticmethod
     def _check(ms):
