@@ -159,7 +159,7 @@ def test_tiled_integer_coded_reassembly(H, W, T):
 
 
 @pytest.mark.parametrize("shape", [(6, 10), (10, 6), (16, 16), (5, 40), (1, 9)])
-@pytest.mark.parametrize("restart", [(), (3,), (2, 4)])
+@pytest.mark.parametrize("restart", [(), (3,), (2, 4), (2, 3), (1,), (1, 2, 3, 4, 5), (9,)])
 def test_gram_ns_equals_standard_ns(shape, restart):
     X = inputs.gaussian(shape, seed=shape[0] * 7 + shape[1])
     g = oracle.gram_ns(X, C5, restart=restart)
