@@ -56,8 +56,12 @@ int main(void) {
   CHECK(himuon_ns_static(mats, mats, 2, NULL, &p, NULL) == HIMUON_ERR_UNSUPPORTED);
   p.tiles = NULL;
 
-  /* argument errors come back before anything touches a device */
+  /* argument errors come back before anything touches a device; an empty
+     call (no matrices) is one of them */
   CHECK(himuon_ns_tiled(NULL, mats, 1, NULL, &p, NULL, 0, NULL) == HIMUON_ERR_INVALID);
+  CHECK(himuon_ns_tiled(mats, mats, 0, NULL, &p, NULL, 0, NULL) == HIMUON_ERR_INVALID);
+  CHECK(himuon_workspace_size(mats, 0, NULL, &p, HIMUON_OP_NS_TILED) == HIMUON_ERR_INVALID);
+  CHECK(himuon_plan_tiles(mats, 0, NULL, 128, records, 16) == HIMUON_ERR_INVALID);
   p.steps = 17;
   CHECK(himuon_ns_tiled(mats, mats, 1, NULL, &p, NULL, 0, NULL) == HIMUON_ERR_UNSUPPORTED);
   p.steps = 5;
