@@ -10,7 +10,8 @@ inputs to float64 and walks the split/tile structure:
 
 * ``ns_map``       -- Algorithm 1 of the "Gram Newton-Schulz" page (sec. 3).
 * ``ns_tiled``     -- the HiMuon tiling ("Hierarchical Muon", abstract).
-* ``gram_ns``      -- Algorithm 3 of the "Gram Newton-Schulz" page (sec. 6).
+* ``gram_ns``      -- Gram NS of the "Gram Newton-Schulz" page (sec. 5-6): the
+  same map computed through the Gram matrix, with restarts.
 * ``split_blocks`` -- the CMuon split of a fused tensor into its functional
   blocks (CMuon article).
 * ``momentum_step`` -- the Muon recap update (sec. 3):
@@ -53,11 +54,12 @@ def _load():
         lib = ctypes.CDLL(build())
         dp = ctypes.POINTER(ctypes.c_double)
         i64, ci = ctypes.c_int64, ctypes.c_int
-        lib.oracle_ns_map.argtypes = [dp, i64, i64, i64, ci, dp, ctypes.c_double, dp, i64]
+        cd = ctypes.c_double
+        lib.oracle_ns_map.argtypes = [dp, i64, i64, i64, ci, dp, cd, cd, dp, i64]
         lib.oracle_ns_map.restype = ci
-        lib.oracle_ns_tiled.argtypes = [dp, i64, i64, i64, i64, ci, dp, ctypes.c_double, dp, i64]
+        lib.oracle_ns_tiled.argtypes = [dp, i64, i64, i64, i64, ci, dp, cd, cd, dp, i64]
         lib.oracle_ns_tiled.restype = ci
-        lib.oracle_gram_ns.argtypes = [dp, i64, i64, i64, ci, dp, ctypes.c_double,
+        lib.oracle_gram_ns.argtypes = [dp, i64, i64, i64, ci, dp, cd, cd,
                                        ctypes.POINTER(ctypes.c_int), ci, dp, i64]
         lib.oracle_gram_ns.restype = ci
         lib.oracle_num_threads.restype = ci
@@ -87,55 +89,59 @@ def _coeffs(coeffs, K: int | None = None) -> tuple[np.ndarray, int]:
     return np.ascontiguousarray(c), c.shape[0]
 
 
-def ns_map(x, coeffs, K: int | None = None, eps: float = EPS) -> np.ndarray:
-    """Standard NS (Algorithm 1) of one matrix, in fp64."""
+def ns_map(x, coeffs, K: int | None = None, eps: float = EPS, safety: float = 1.0) -> np.ndarray:
+    """Standard NS (Algorithm 1) of one matrix, in fp64.  ``safety`` divides the
+    normalised input (sec. 6 implementation notes; 1.0 = off)."""
     X = _f64(x)
     c, K = _coeffs(coeffs, K)
     h, w = X.shape
     out = np.zeros((h, w), dtype=np.float64)
-    rc = _load().oracle_ns_map(_ptr(X), w, h, w, K, _ptr(c), eps, _ptr(out), w)
+    rc = _load().oracle_ns_map(_ptr(X), w, h, w, K, _ptr(c), eps, float(safety), _ptr(out), w)
     if rc != 0:
         raise MemoryError("oracle_ns_map failed")
     return out
 
 
-def ns_tiled(x, T: int, coeffs, K: int | None = None, eps: float = EPS) -> np.ndarray:
+def ns_tiled(x, T: int, coeffs, K: int | None = None, eps: float = EPS, safety: float = 1.0) -> np.ndarray:
     """HiMuon: NS applied to each T x T tile (ragged edges smaller), in place."""
     X = _f64(x)
     c, K = _coeffs(coeffs, K)
     H, W = X.shape
     out = np.zeros((H, W), dtype=np.float64)
-    rc = _load().oracle_ns_tiled(_ptr(X), W, H, W, int(T), K, _ptr(c), eps, _ptr(out), W)
+    rc = _load().oracle_ns_tiled(_ptr(X), W, H, W, int(T), K, _ptr(c), eps, float(safety), _ptr(out), W)
     if rc != 0:
         raise RuntimeError(f"oracle_ns_tiled failed ({rc})")
     return out
 
 
-def gram_ns(x, coeffs, K: int | None = None, restart: Sequence[int] = (3,), eps: float = EPS) -> np.ndarray:
-    """Stabilised Gram NS (Algorithm 3) of one matrix; restart steps are 1-based."""
+def gram_ns(x, coeffs, K: int | None = None, restart: Sequence[int] = (3,), eps: float = EPS,
+            safety: float = 1.0) -> np.ndarray:
+    """Gram NS of one matrix (sec. 5-6): R = X X^T, Q = I, per step P = p_t(R),
+    Q <- P Q, R <- P R P; output Q X.  ``restart`` lists the 1-based steps
+    before which X <- Q X, R <- X X^T, Q <- I."""
     X = _f64(x)
     c, K = _coeffs(coeffs, K)
     h, w = X.shape
     out = np.zeros((h, w), dtype=np.float64)
     rs = (ctypes.c_int * max(1, len(restart)))(*restart)
-    rc = _load().oracle_gram_ns(_ptr(X), w, h, w, K, _ptr(c), eps, rs, len(restart), _ptr(out), w)
+    rc = _load().oracle_gram_ns(_ptr(X), w, h, w, K, _ptr(c), eps, float(safety), rs, len(restart), _ptr(out), w)
     if rc != 0:
         raise MemoryError("oracle_gram_ns failed")
     return out
 
 
 def gram_ns_tiled(x, T: int, coeffs, K: int | None = None, restart: Sequence[int] = (3,),
-                  eps: float = EPS) -> np.ndarray:
+                  eps: float = EPS, safety: float = 1.0) -> np.ndarray:
     """Gram NS applied to each T x T tile ("Hierarchical Muon" abstract: the
     same map per tile, reassembled; ragged edge tiles smaller).  T <= 0 or at
     least the matrix's sides: the whole matrix."""
     X = _f64(x)
     H, W = X.shape
     if T <= 0 or T >= max(H, W):
-        return gram_ns(X, coeffs, K, restart, eps)
+        return gram_ns(X, coeffs, K, restart, eps, safety)
     out = np.zeros((H, W), dtype=np.float64)
     for r0, c0, h, w in tile_grid(H, W, T):
-        out[r0:r0 + h, c0:c0 + w] = gram_ns(X[r0:r0 + h, c0:c0 + w], coeffs, K, restart, eps)
+        out[r0:r0 + h, c0:c0 + w] = gram_ns(X[r0:r0 + h, c0:c0 + w], coeffs, K, restart, eps, safety)
     return out
 
 
@@ -160,12 +166,13 @@ def split_blocks(shape: tuple[int, int], split: tuple[int, Sequence[int]] | None
     return blocks
 
 
-def ns_tiled_split(x, T: int, coeffs, K: int | None = None, split=None, eps: float = EPS) -> np.ndarray:
+def ns_tiled_split(x, T: int, coeffs, K: int | None = None, split=None, eps: float = EPS,
+                   safety: float = 1.0) -> np.ndarray:
     """Split (CMuon) then tile (HiMuon) each block; blocks are independent."""
     X = _f64(x)
     out = np.zeros_like(X)
     for (r0, c0, h, w) in split_blocks(X.shape, split):
-        out[r0:r0 + h, c0:c0 + w] = ns_tiled(X[r0:r0 + h, c0:c0 + w], T, coeffs, K, eps)
+        out[r0:r0 + h, c0:c0 + w] = ns_tiled(X[r0:r0 + h, c0:c0 + w], T, coeffs, K, eps, safety)
     return out
 
 
@@ -176,10 +183,10 @@ def momentum(M, G, mu: float) -> np.ndarray:
 
 
 def momentum_step(W, M, G, mu: float, eta: float, T: int, coeffs, K: int | None = None,
-                  split=None, eps: float = EPS):
+                  split=None, eps: float = EPS, safety: float = 1.0):
     """One Muon step with tiled NS: returns (W', M', O) in fp64."""
     Mp = momentum(M, G, mu)
-    O = ns_tiled_split(Mp, T, coeffs, K, split, eps)
+    O = ns_tiled_split(Mp, T, coeffs, K, split, eps, safety)
     eta = float(np.float32(eta))
     return _f64(W) - eta * O, Mp, O
 

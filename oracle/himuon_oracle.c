@@ -16,10 +16,15 @@
  *  - same page, sec. 3, Algorithm 1 (standard Newton-Schulz): normalise by
  *      (||X||_F + eps), transpose when the input is taller than wide, then per
  *      step A = X X^T, B = b_t A + c_t A^2, X = a_t X + B X, undo the transpose.
- *  - same page, sec. 6, Algorithm 3 (stabilised Gram Newton-Schulz):
- *      R = X X^T, Q = I; per step (with a restart X <- Q X, R <- X X^T, Q <- I
- *      before the listed steps) Z = b R + c R^2, Q <- Q Z + a Q,
- *      RZ <- R Z + a R, R <- Z RZ + a RZ; output Q X.
+ *  - same page, sec. 2 and 5-6 (Gram Newton-Schulz): one NS step is
+ *      X_t = p_t(R_{t-1}) X_{t-1} with R = X X^T and the step polynomial
+ *      p_t(R) = a_t I + b_t R + c_t R^2, so after t steps X_t = Q_t X_0 with
+ *      Q_t = p_t(R_{t-1}) Q_{t-1}, and the Gram matrix evolves as
+ *      R_t = p_t(R_{t-1}) R_{t-1} p_t(R_{t-1}); the method tracks R and Q and
+ *      forms X only at the end (or at a restart, which materialises X = Q X,
+ *      recomputes R from it and starts Q again from I).
+ *  - same page, sec. 6, implementation notes: the optional safety factor
+ *      divides the normalised input (the example given is 1.05).
  *  - "Hierarchical Muon: Tiled Newton-Schulz Updates", abstract: cut the
  *      matrix into T x T tiles, apply the same NS map to each tile on its own,
  *      put the results back in place.
@@ -77,11 +82,12 @@ static double frobenius(const double *X, int64_t count) {
 
 /*
  * Algorithm 1 (standard NS) on one h x w matrix x (row-major, leading dim ldx).
- * coeffs holds K triples (a_t, b_t, c_t).  Result to out (leading dim ldo).
+ * coeffs holds K triples (a_t, b_t, c_t).  The normalised input is divided by
+ * `safety` (1 = off).  Result to out (leading dim ldo).
  * Returns 0, or -1 on allocation failure.
  */
 int oracle_ns_map(const double *x, int64_t ldx, int64_t h, int64_t w, int K,
-                  const double *coeffs, double eps, double *out, int64_t ldo) {
+                  const double *coeffs, double eps, double safety, double *out, int64_t ldo) {
   if (h <= 0 || w <= 0) return 0;
   const int tr = h > w;              /* "If m < n: X <- X^T" for an n x m input */
   const int64_t n = tr ? w : h;      /* rows of the iterate, n <= m */
@@ -99,9 +105,9 @@ int oracle_ns_map(const double *x, int64_t ldx, int64_t h, int64_t w, int K,
   /* copy the input as an h x w dense block */
   for (int64_t i = 0; i < h; ++i)
     for (int64_t j = 0; j < w; ++j) Y[i * w + j] = x[i * ldx + j];
-  /* X <- X / (||X||_F + eps) */
+  /* X <- X / (||X||_F + eps), then X <- X / safety */
   const double nrm = frobenius(Y, h * w);
-  for (int64_t i = 0; i < h * w; ++i) Y[i] = Y[i] / (nrm + eps);
+  for (int64_t i = 0; i < h * w; ++i) Y[i] = Y[i] / (nrm + eps) / safety;
   if (tr) transpose(Y, X, h, w); else memcpy(X, Y, sizeof(double) * n * m);
   for (int t = 0; t < K; ++t) {
     const double a = coeffs[3 * t + 0], b = coeffs[3 * t + 1], c = coeffs[3 * t + 2];
@@ -124,7 +130,7 @@ int oracle_ns_map(const double *x, int64_t ldx, int64_t h, int64_t w, int K,
  * on its own and is written back in place.  T >= max(H, W) is full-matrix NS.
  */
 int oracle_ns_tiled(const double *in, int64_t ldi, int64_t H, int64_t W, int64_t T, int K,
-                    const double *coeffs, double eps, double *out, int64_t ldo) {
+                    const double *coeffs, double eps, double safety, double *out, int64_t ldo) {
   if (T <= 0) return -2;
   const int64_t tr = (H + T - 1) / T, tc = (W + T - 1) / T;
   int err = 0;
@@ -134,61 +140,74 @@ int oracle_ns_tiled(const double *in, int64_t ldi, int64_t H, int64_t W, int64_t
     const int64_t r0 = p * T, c0 = q * T;
     const int64_t h = (H - r0 < T) ? H - r0 : T;
     const int64_t w = (W - c0 < T) ? W - c0 : T;
-    err |= oracle_ns_map(in + r0 * ldi + c0, ldi, h, w, K, coeffs, eps, out + r0 * ldo + c0, ldo);
+    err |= oracle_ns_map(in + r0 * ldi + c0, ldi, h, w, K, coeffs, eps, safety, out + r0 * ldo + c0, ldo);
   }
   return err ? -1 : 0;
 }
 
+/* P = a I + b R + c R^2 (n x n), the step polynomial of the Gram matrix R. */
+static void step_polynomial(const double *R, double a, double b, double c, double *P, double *tmp, int64_t n) {
+  mm_ab(R, R, tmp, n, n, n);
+  for (int64_t i = 0; i < n * n; ++i) P[i] = b * R[i] + c * tmp[i] + ((i / n == i % n) ? a : 0.0);
+}
+
+static void set_identity(double *Q, int64_t n) {
+  for (int64_t i = 0; i < n * n; ++i) Q[i] = (i / n == i % n) ? 1.0 : 0.0;
+}
+
 /*
- * Algorithm 3 (stabilised Gram NS) on one h x w matrix.  restart[] lists the
- * 1-based step indices t before which X <- Q X, R <- X X^T, Q <- I happens
- * (the page restarts at t = 3).  With n_restart = 0 this is Algorithm 2 with
- * the identity term added explicitly, which is the same map.
+ * Gram NS on one h x w matrix: the NS map computed through the Gram matrix.
+ * Normalise (and divide by `safety`) and transpose exactly as in Algorithm 1;
+ * then R = X X^T and Q = I, and per step t, with P = p_t(R):
+ *     Q <- P Q          (the accumulated left factor: X_t = Q X_0)
+ *     R <- P R P        (the Gram matrix of X_t)
+ * and the output is Q X.  restart[] lists the 1-based steps t before which
+ * the current iterate is materialised (X <- Q X), its Gram matrix recomputed
+ * (R <- X X^T) and Q started again from I; the page restarts before t = 3.
+ * In exact arithmetic every restart leaves the result unchanged.
  */
 int oracle_gram_ns(const double *x, int64_t ldx, int64_t h, int64_t w, int K, const double *coeffs,
-                   double eps, const int *restart, int n_restart, double *out, int64_t ldo) {
+                   double eps, double safety, const int *restart, int n_restart, double *out, int64_t ldo) {
   if (h <= 0 || w <= 0) return 0;
   const int tr = h > w;
   const int64_t n = tr ? w : h, m = tr ? h : w;
   double *X = malloc(sizeof(double) * n * m), *Y = malloc(sizeof(double) * n * m);
   double *R = malloc(sizeof(double) * n * n), *Q = malloc(sizeof(double) * n * n);
-  double *Z = malloc(sizeof(double) * n * n), *R2 = malloc(sizeof(double) * n * n);
-  double *RZ = malloc(sizeof(double) * n * n), *T1 = malloc(sizeof(double) * n * n);
-  if (!X || !Y || !R || !Q || !Z || !R2 || !RZ || !T1) {
-    free(X); free(Y); free(R); free(Q); free(Z); free(R2); free(RZ); free(T1);
+  double *P = malloc(sizeof(double) * n * n), *T1 = malloc(sizeof(double) * n * n);
+  double *T2 = malloc(sizeof(double) * n * n);
+  if (!X || !Y || !R || !Q || !P || !T1 || !T2) {
+    free(X); free(Y); free(R); free(Q); free(P); free(T1); free(T2);
     return -1;
   }
   for (int64_t i = 0; i < h; ++i)
     for (int64_t j = 0; j < w; ++j) Y[i * w + j] = x[i * ldx + j];
   const double nrm = frobenius(Y, h * w);
-  for (int64_t i = 0; i < h * w; ++i) Y[i] = Y[i] / (nrm + eps);
+  for (int64_t i = 0; i < h * w; ++i) Y[i] = Y[i] / (nrm + eps) / safety;
   if (tr) transpose(Y, X, h, w); else memcpy(X, Y, sizeof(double) * n * m);
-  mm_abt(X, X, R, n, n, m);                                   /* R_0 = X X^T */
-  for (int64_t i = 0; i < n * n; ++i) Q[i] = (i / n == i % n) ? 1.0 : 0.0;   /* Q_0 = I */
+  mm_abt(X, X, R, n, n, m);
+  set_identity(Q, n);
   for (int t = 1; t <= K; ++t) {
-    const double a = coeffs[3 * (t - 1) + 0], b = coeffs[3 * (t - 1) + 1], c = coeffs[3 * (t - 1) + 2];
     int is_restart = 0;
     for (int r = 0; r < n_restart; ++r) is_restart |= (restart[r] == t);
     if (is_restart) {
-      mm_ab(Q, X, Y, n, m, n);                                /* X <- Q X    */
+      mm_ab(Q, X, Y, n, m, n);
       memcpy(X, Y, sizeof(double) * n * m);
-      mm_abt(X, X, R, n, n, m);                               /* R <- X X^T  */
-      for (int64_t i = 0; i < n * n; ++i) Q[i] = (i / n == i % n) ? 1.0 : 0.0;
+      mm_abt(X, X, R, n, n, m);
+      set_identity(Q, n);
     }
-    mm_ab(R, R, R2, n, n, n);
-    for (int64_t i = 0; i < n * n; ++i) Z[i] = b * R[i] + c * R2[i];           /* Z = bR + cR^2   */
-    mm_ab(Q, Z, T1, n, n, n);
-    for (int64_t i = 0; i < n * n; ++i) Q[i] = T1[i] + a * Q[i];               /* Q = QZ + aQ     */
-    mm_ab(R, Z, T1, n, n, n);
-    for (int64_t i = 0; i < n * n; ++i) RZ[i] = T1[i] + a * R[i];              /* RZ = RZ + aR    */
-    mm_ab(Z, RZ, T1, n, n, n);
-    for (int64_t i = 0; i < n * n; ++i) R[i] = T1[i] + a * RZ[i];              /* R = Z RZ + a RZ */
+    const double *ct = coeffs + 3 * (t - 1);
+    step_polynomial(R, ct[0], ct[1], ct[2], P, T1, n);
+    mm_ab(P, Q, T1, n, n, n);                 /* Q <- P Q   */
+    memcpy(Q, T1, sizeof(double) * n * n);
+    mm_ab(P, R, T1, n, n, n);                 /* R <- P R P */
+    mm_ab(T1, P, T2, n, n, n);
+    memcpy(R, T2, sizeof(double) * n * n);
   }
-  mm_ab(Q, X, Y, n, m, n);                                    /* output Q X  */
+  mm_ab(Q, X, Y, n, m, n);
   if (tr) { transpose(Y, X, n, m); memcpy(Y, X, sizeof(double) * n * m); }
   for (int64_t i = 0; i < h; ++i)
     for (int64_t j = 0; j < w; ++j) out[i * ldo + j] = Y[i * w + j];
-  free(X); free(Y); free(R); free(Q); free(Z); free(R2); free(RZ); free(T1);
+  free(X); free(Y); free(R); free(Q); free(P); free(T1); free(T2);
   return 0;
 }
 

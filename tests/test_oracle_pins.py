@@ -37,11 +37,11 @@ def phi(x, coeffs):
     return x
 
 
-def ns_by_svd(X, coeffs, eps=EPS):
-    """The SVD route: U phi(sigma / (||X||_F + eps)) V^T."""
+def ns_by_svd(X, coeffs, eps=EPS, safety=1.0):
+    """The SVD route: U phi(sigma / (safety (||X||_F + eps))) V^T."""
     U, s, Vt = np.linalg.svd(X, full_matrices=False)
     nrm = np.sqrt(np.sum(X * X))
-    return (U * phi(s / (nrm + eps), coeffs)[None, :]) @ Vt
+    return (U * phi(s / ((nrm + eps) * safety), coeffs)[None, :]) @ Vt
 
 
 def rel(a, b):
@@ -77,6 +77,40 @@ def test_eps_sits_beside_the_norm():
     out = oracle.ns_map(X, CFG * 5)
     assert rel(out, ns_by_svd(X, CFG * 5)) < 1e-11
     assert rel(out, ns_by_svd(X, CFG * 5, eps=0.0)) > 1e-3
+
+
+@pytest.mark.parametrize("shape", [(3, 5), (6, 6), (9, 4)])
+@pytest.mark.parametrize("safety", [1.05, 2.0])
+def test_safety_factor_divides_the_normalised_input(shape, safety):
+    """"Gram Newton-Schulz" page, sec. 6 implementation notes: the input is
+    divided by the safety factor (1.05 in the example) after normalisation, so
+    the singular values entering phi are sigma / (safety (||X||_F + eps))."""
+    X = inputs.gaussian(shape, seed=shape[0] + 17 * shape[1])
+    for co in (C5, C5[:2]):
+        out = oracle.ns_map(X, co, safety=safety)
+        assert rel(out, ns_by_svd(X, co, safety=safety)) < 1e-11
+        g = oracle.gram_ns(X, co, restart=(2,), safety=safety)
+        assert rel(g, ns_by_svd(X, co, safety=safety)) < 1e-10
+        t = oracle.ns_tiled(X, 2, co, safety=safety)
+        for r0, c0, h, w in oracle.tile_grid(*shape, 2):
+            blk = X[r0:r0 + h, c0:c0 + w]
+            assert rel(t[r0:r0 + h, c0:c0 + w], ns_by_svd(blk, co, safety=safety)) < 1e-11
+    # two steps leave the factor visible (five converged steps nearly hide it)
+    out = oracle.ns_map(X, C5[:2], safety=safety)
+    assert rel(out, ns_by_svd(X, C5[:2])) > 1e-3                       # the factor is applied
+    assert rel(out, ns_by_svd(X, C5[:2], safety=1.0 / safety)) > 1e-3  # ... as a divisor
+
+
+def test_safety_factor_scales_norm_plus_eps():
+    # ||X||_F ~ 1e-6: dividing (||X||_F + eps) by the factor and dividing
+    # ||X||_F alone before adding eps give visibly different results.
+    X = inputs.gaussian((4, 7), seed=12)
+    X = X / np.linalg.norm(X) * 1e-6
+    out = oracle.ns_map(X, CFG * 5, safety=2.0)
+    assert rel(out, ns_by_svd(X, CFG * 5, safety=2.0)) < 1e-11
+    U, sv, Vt = np.linalg.svd(X, full_matrices=False)
+    other = (U * phi(sv / (2.0 * np.linalg.norm(X) + EPS), CFG * 5)[None, :]) @ Vt
+    assert rel(out, other) > 1e-3
 
 
 @pytest.mark.parametrize("x", [2.5, -0.3, 1e-9, -7.0])
