@@ -221,11 +221,14 @@ HIMUON_API int himuon_version(void);
  * in bf16 and 1024 x 1024 in fp32.
  *
  * The first call on a device looks up that device's address of the array
- * (cudaGetSymbolAddress, with the device current); make that first call before
- * any stream capture.  All calls share the one array and it keeps the last
- * call's contents: calls that overlap on the GPU (on different streams, or
- * from different host threads) race on it and must be serialised by the
- * caller.  Calls on one stream are ordered and safe.
+ * (cudaGetSymbolAddress, with the device current) and keeps it for later
+ * calls; make that first call before any stream capture.  A cudaDeviceReset
+ * of that device invalidates the kept address: do not call himuon_ns_static
+ * after resetting a device it was used on.  Thin tiles (short side <= 64) of
+ * a bf16 call run in fp32, as on the workspace path.  All calls share the one
+ * array and it keeps the last call's contents: calls that overlap on the GPU
+ * (on different streams, or from different host threads) race on it and must
+ * be serialised by the caller.  Calls on one stream are ordered and safe.
  */
 #define HIMUON_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 HIMUON_API int himuon_ns_static(const himuon_mat *in, const himuon_mat *out, int32_t n, const himuon_split *splits,

@@ -70,6 +70,24 @@ def test_static_scratch_matches_workspace_path_twice(hm):
     assert hm.device_status() == 0
 
 
+def test_static_scratch_fp32_matches_workspace_path(hm):
+    """An fp32 call (CUDA-core path, its own workspace layout): 256 x 512 at
+    T = 256 and full NS, against the workspace entry points within the fp32
+    path's tolerance (1e-4 per-tile relative Frobenius error)."""
+    x = torch.from_numpy(inputs.gaussian((256, 512), seed=44)).to("cuda", torch.float32)
+    for T in (256, 0):
+        p = hm.params(T, inputs.QUINTIC, steps=5, compute=hm.FP32)
+        ref = torch.empty_like(x)
+        (hm.ns_tiled if T > 0 else hm.ns_full)([x], [ref], p)
+        got = torch.full_like(x, float("nan"))
+        assert hm.ns_static([x], [got], p) == 0
+        torch.cuda.synchronize()
+        a, b = got.double().cpu().numpy(), ref.double().cpu().numpy()
+        assert np.all(np.isfinite(a))
+        assert per_tile_errors(a, b, T).max() <= 1e-4
+    assert hm.device_status() == 0
+
+
 def test_static_scratch_refuses_oversized_calls(hm):
     x = torch.zeros(4096, 4096, device="cuda", dtype=torch.bfloat16)
     out = torch.zeros_like(x)

@@ -15,6 +15,7 @@
 #include <mutex>
 #include <memory>
 #include <string>
+#include <tuple>
 #include <vector>
 
 #include "himuon.h"
@@ -165,6 +166,7 @@ enum PathKind { kPathResident = 0, kPathStaged = 1 };
 struct TileClass {
   int64_t n, m;          // padded iterate shape (n <= m)
   bool padded;           // some tile of the class is smaller than n x m
+  bool thin;             // every tile of the class has a short side <= kThinSide
   std::vector<DevTile> tiles;
   int64_t dev_offset;    // index of the class's first DevTile in the device table
 };
@@ -297,6 +299,55 @@ PlanCache &cache() {
   return *c;
 }
 
+// Tiles whose short side is at most this are "thin": rounding their operands
+// to bf16's 8 significant bits moves their output singular values by up to
+// ~0.1 (a 16-bit operand type with 11 bits keeps them near 0.01).
+constexpr int64_t kThinSide = 64;
+
+// Staged tile classes: tiles grouped by padded iterate shape (n, m), n <= m
+// (multiples of 128, tall tiles transposed), thin tiles in classes of their own.
+void staged_classes(const std::vector<HostBlock> &blocks, std::vector<TileClass> &classes) {
+  std::map<std::tuple<int64_t, int64_t, bool>, size_t> cls;
+  for (size_t bi = 0; bi < blocks.size(); ++bi) {
+    const HostBlock &b = blocks[bi];
+    for (int64_t tr = 0; tr < b.tiles_r; ++tr)
+      for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
+        DevTile t;
+        t.block = static_cast<int32_t>(bi);
+        t.r0 = static_cast<int32_t>(tr * b.T);
+        t.c0 = static_cast<int32_t>(tc * b.T);
+        t.h = static_cast<int32_t>(std::min(b.T, b.rows - t.r0));
+        t.w = static_cast<int32_t>(std::min(b.T, b.cols - t.c0));
+        t.transposed = t.h > t.w ? 1 : 0;
+        const int64_t n = round_up(std::min(t.h, t.w), 128), m = round_up(std::max(t.h, t.w), 128);
+        const bool thin = std::min(t.h, t.w) <= kThinSide;
+        const auto key = std::make_tuple(n, m, thin);
+        auto it = cls.find(key);
+        if (it == cls.end()) {
+          it = cls.emplace(key, classes.size()).first;
+          TileClass c;
+          c.n = n;
+          c.m = m;
+          c.padded = false;
+          c.thin = thin;
+          classes.push_back(c);
+        }
+        TileClass &c = classes[it->second];
+        if (std::min(t.h, t.w) != n || std::max(t.h, t.w) != m) c.padded = true;
+        c.tiles.push_back(t);
+      }
+  }
+}
+
+// Arithmetic of a staged class.  A bf16 call runs Gram NS with fp16 operands
+// (the Gram Newton-Schulz page prescribes fp16 over bf16 for it), and thin
+// tiles of standard NS in fp32 on the CUDA cores; otherwise as asked.
+int class_compute(const TileClass &c, int op, int compute) {
+  if (compute != HIMUON_BF16) return compute;
+  if (op == HIMUON_OP_GRAM_NS) return HIMUON_FP16;
+  return c.thin ? HIMUON_FP32 : HIMUON_BF16;
+}
+
 int build_plan(int device, int op, const CallMats &cm, const himuon_split *splits, const himuon_ns_params &p,
                std::shared_ptr<Plan> &out) {
   auto plan = std::make_shared<Plan>();
@@ -339,35 +390,7 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
   }
   std::vector<DevTile> dtiles;
   if (!resident) {
-    // shape classes of the staged path: padded (n, m), n <= m, multiples of 128
-    std::map<std::pair<int64_t, int64_t>, size_t> cls;
-    for (size_t bi = 0; bi < plan->blocks.size(); ++bi) {
-      const HostBlock &b = plan->blocks[bi];
-      for (int64_t tr = 0; tr < b.tiles_r; ++tr)
-        for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
-          DevTile t;
-          t.block = static_cast<int32_t>(bi);
-          t.r0 = static_cast<int32_t>(tr * b.T);
-          t.c0 = static_cast<int32_t>(tc * b.T);
-          t.h = static_cast<int32_t>(std::min(b.T, b.rows - t.r0));
-          t.w = static_cast<int32_t>(std::min(b.T, b.cols - t.c0));
-          t.transposed = t.h > t.w ? 1 : 0;
-          const int64_t n = round_up(std::min(t.h, t.w), 128), m = round_up(std::max(t.h, t.w), 128);
-          auto key = std::make_pair(n, m);
-          auto it = cls.find(key);
-          if (it == cls.end()) {
-            it = cls.emplace(key, plan->classes.size()).first;
-            TileClass c;
-            c.n = n;
-            c.m = m;
-            c.padded = false;
-            plan->classes.push_back(c);
-          }
-          TileClass &c = plan->classes[it->second];
-          if (std::min(t.h, t.w) != n || std::max(t.h, t.w) != m) c.padded = true;
-          c.tiles.push_back(t);
-        }
-    }
+    staged_classes(plan->blocks, plan->classes);
     for (TileClass &c : plan->classes) {
       c.dev_offset = static_cast<int64_t>(dtiles.size());
       dtiles.insert(dtiles.end(), c.tiles.begin(), c.tiles.end());
@@ -392,8 +415,8 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
             resident ? "resident" : "staged", plan->blocks.size(), (long long)plan->n_tiles, plan->classes.size(),
             tmaps.size());
     for (const TileClass &c : plan->classes)
-      fprintf(stderr, "[himuon]   class n=%lld m=%lld tiles=%zu padded=%d\n", (long long)c.n, (long long)c.m,
-              c.tiles.size(), (int)c.padded);
+      fprintf(stderr, "[himuon]   class n=%lld m=%lld tiles=%zu padded=%d thin=%d compute=%d\n", (long long)c.n,
+              (long long)c.m, c.tiles.size(), (int)c.padded, (int)c.thin, class_compute(c, op, p.compute));
   }
   out = plan;
   return HIMUON_OK;
@@ -497,10 +520,12 @@ int64_t chunk_tiles(const TileClass &c, size_t limit, int compute, bool gram) {
   return k;
 }
 
-int64_t staged_ws_bytes(const Plan &plan, int compute, bool gram) {
+int64_t staged_ws_bytes(const Plan &plan, int op, int compute) {
+  const bool gram = op == HIMUON_OP_GRAM_NS;
   int64_t need = 0;
   for (const TileClass &c : plan.classes)
-    need = std::max<int64_t>(need, static_cast<int64_t>(ws_layout(c.n, c.m, 1, compute, gram).total));
+    need = std::max<int64_t>(need,
+                             static_cast<int64_t>(ws_layout(c.n, c.m, 1, class_compute(c, op, compute), gram).total));
   return need;
 }
 
@@ -548,14 +573,14 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
                cudaStream_t stream) {
   const bool gram = op == HIMUON_OP_GRAM_NS;
   const bool step = op == HIMUON_OP_MOMENTUM_STEP;
-  const int compute = p.compute;
-  const bool f32 = compute == HIMUON_FP32;
   const size_t limit = chunk_limit(ws_bytes, p);
-  Ops ops{compute, compute == HIMUON_FP16 ? HIMUON_FP16 : HIMUON_BF16, status_ptr(), stream};
-  const int32_t dt16 = ops.op16;
   const float safety = p.safety > 0.f ? p.safety : 1.f;
   char *W = static_cast<char *>(ws);
   for (const TileClass &c : plan.classes) {
+    const int compute = class_compute(c, op, p.compute);
+    const bool f32 = compute == HIMUON_FP32;
+    Ops ops{compute, compute == HIMUON_FP16 ? HIMUON_FP16 : HIMUON_BF16, status_ptr(), stream};
+    const int32_t dt16 = ops.op16;
     const int64_t per = chunk_tiles(c, limit, compute, gram);
     if (per < 1) return HIMUON_ERR_WORKSPACE;
     const int64_t n = c.n, m = c.m;
@@ -737,6 +762,7 @@ int run_resident(const Plan &plan, int op, const himuon_ns_params &p, float mu, 
   a.has_w = has_w ? 1 : 0;
   a.has_o = has_o ? 1 : 0;
   a.op_fmt = p.compute == HIMUON_FP16 ? 0 : 1;
+  a.f16_small = p.compute == HIMUON_BF16 ? 1 : 0;
   a.mu = mu;
   a.lr = lr;
   a.eps = p.eps;
@@ -785,7 +811,7 @@ int prepare(int op, const CallMats &cm, const himuon_split *splits, const himuon
   pr.has_w = op == HIMUON_OP_MOMENTUM_STEP && cm.role[kRoleW];
   pr.has_o = cm.role[kRoleOut] != nullptr;
   if (pr.plan->path == kPathResident) return HIMUON_OK;
-  const int64_t need = staged_ws_bytes(*pr.plan, p->compute, op == HIMUON_OP_GRAM_NS);
+  const int64_t need = staged_ws_bytes(*pr.plan, op, p->compute);
   if (!ws || static_cast<int64_t>(ws_bytes) < need) return HIMUON_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return HIMUON_ERR_ALIGNMENT;
   return HIMUON_OK;
@@ -884,21 +910,15 @@ int64_t workspace_one(const CallMats &cm, const himuon_split *splits, const himu
   // staged: one tile of the largest class is the minimum; a full chunk of every
   // class makes the call run in one chunk per class.
   int64_t need = 0;
-  std::map<std::pair<int64_t, int64_t>, int64_t> counts;
-  for (const HostBlock &b : blocks)
-    for (int64_t tr = 0; tr < b.tiles_r; ++tr)
-      for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
-        const int64_t h = std::min(b.T, b.rows - tr * b.T), w = std::min(b.T, b.cols - tc * b.T);
-        counts[{round_up(std::min(h, w), 128), round_up(std::max(h, w), 128)}] += 1;
-      }
-  for (auto &kv : counts) {
-    int64_t k = std::min<int64_t>(kv.second, 65535);
-    int64_t bytes = static_cast<int64_t>(ws_layout(kv.first.first, kv.first.second, k, p.compute,
-                                                   op == HIMUON_OP_GRAM_NS).total);
+  std::vector<TileClass> classes;
+  staged_classes(blocks, classes);
+  const bool gram = op == HIMUON_OP_GRAM_NS;
+  for (const TileClass &c : classes) {
+    const int compute = class_compute(c, op, p.compute);
+    int64_t k = std::min<int64_t>(static_cast<int64_t>(c.tiles.size()), 65535);
+    int64_t bytes = static_cast<int64_t>(ws_layout(c.n, c.m, k, compute, gram).total);
     if (p.chunk_bytes > 0 && bytes > p.chunk_bytes)
-      bytes = std::max<int64_t>(p.chunk_bytes, static_cast<int64_t>(ws_layout(kv.first.first, kv.first.second, 1,
-                                                                                p.compute, op == HIMUON_OP_GRAM_NS)
-                                                                          .total));
+      bytes = std::max<int64_t>(p.chunk_bytes, static_cast<int64_t>(ws_layout(c.n, c.m, 1, compute, gram).total));
     need = std::max(need, bytes);
   }
   return need;
@@ -950,33 +970,7 @@ int run_staged_into(int op, const himuon_mat *in, const himuon_mat *out, int32_t
       d.dtype[r] = m.dtype;
     }
   }
-  std::map<std::pair<int64_t, int64_t>, size_t> cls;
-  for (size_t bi = 0; bi < plan.blocks.size(); ++bi) {
-    const HostBlock &b = plan.blocks[bi];
-    for (int64_t tr = 0; tr < b.tiles_r; ++tr)
-      for (int64_t tc = 0; tc < b.tiles_c; ++tc) {
-        DevTile t;
-        t.block = static_cast<int32_t>(bi);
-        t.r0 = static_cast<int32_t>(tr * b.T);
-        t.c0 = static_cast<int32_t>(tc * b.T);
-        t.h = static_cast<int32_t>(std::min(b.T, b.rows - t.r0));
-        t.w = static_cast<int32_t>(std::min(b.T, b.cols - t.c0));
-        t.transposed = t.h > t.w ? 1 : 0;
-        const int64_t nn = round_up(std::min(t.h, t.w), 128), mm = round_up(std::max(t.h, t.w), 128);
-        auto it = cls.find({nn, mm});
-        if (it == cls.end()) {
-          it = cls.emplace(std::make_pair(nn, mm), plan.classes.size()).first;
-          TileClass c;
-          c.n = nn;
-          c.m = mm;
-          c.padded = false;
-          plan.classes.push_back(c);
-        }
-        TileClass &c = plan.classes[it->second];
-        if (std::min(t.h, t.w) != nn || std::max(t.h, t.w) != mm) c.padded = true;
-        c.tiles.push_back(t);
-      }
-  }
+  staged_classes(plan.blocks, plan.classes);
   std::vector<DevTile> dtiles;
   for (TileClass &c : plan.classes) {
     c.dev_offset = static_cast<int64_t>(dtiles.size());
@@ -986,7 +980,7 @@ int run_staged_into(int op, const himuon_mat *in, const himuon_mat *out, int32_t
   const size_t st = round_up(sizeof(DevTile) * dtiles.size(), 256);
   if (sb + st >= scratch_bytes) return HIMUON_ERR_TOO_LARGE;
   const size_t ws_bytes = scratch_bytes - sb - st;
-  if (static_cast<int64_t>(ws_bytes) < staged_ws_bytes(plan, p->compute, false)) return HIMUON_ERR_TOO_LARGE;
+  if (static_cast<int64_t>(ws_bytes) < staged_ws_bytes(plan, op, p->compute)) return HIMUON_ERR_TOO_LARGE;
   char *base = static_cast<char *>(scratch);
   if (cudaMemcpyAsync(base, dblocks.data(), sizeof(DevBlock) * dblocks.size(), cudaMemcpyHostToDevice, stream) !=
           cudaSuccess ||

@@ -43,6 +43,15 @@
 // them), or into D_X while D_X holds nothing live.  Keeping A operands out of
 // shared memory halves the operand traffic there (N = 128 MMAs with both
 // operands in shared memory run at the shared-memory bandwidth limit).
+// Operand type.  The call asks for bf16 or fp16 operands.  A bf16 call still
+// rounds to fp16 the operands of a super-tile whose tiles all have a short
+// side of at most 64 (T = 64 and 32, and ragged edge tiles): rounding the
+// operands of such tiles to bf16's 8 significant bits moves their output
+// singular values by up to ~0.1, where fp16's 11 bits keep them within ~0.01,
+// at the same tensor-core rate.  A tile whose normalised norm is below 2^-10
+// (input norm far below eps) keeps bf16, whose range fp16 lacks.  The choice
+// is made per super-tile at run time, after its norms are known.
+//
 // The momentum update M' = mu M + G is fused into the prologue (M' written
 // back once) and W <- W - lr O into the epilogue, so HBM sees one read and one
 // write per element and role.  The next tile's inputs are loaded (TMA) as soon
@@ -64,20 +73,25 @@ namespace {
 
 constexpr int kGroupWarps = 8;
 constexpr int kGroupThreads = kGroupWarps * 32;
-constexpr int kThreads = 2 * kGroupThreads;
+constexpr int kIssuerWarp = 2 * kGroupWarps;          // warp 16 issues every MMA
+constexpr int kThreads = 2 * kGroupThreads + 32;
 constexpr uint32_t kHalf = 16384;          // one 64-column, 128-row swizzled half tile
 constexpr uint32_t kOffX = 0, kOffS = 32768, kOffW = 65536, kGroupBytes = 98304;
 constexpr uint32_t kOffBars = 2 * kGroupBytes;
 constexpr int kMaxSmemBlocks = 256;        // block tables up to this size live in shared memory
 constexpr int kMaxPack = 4;                // tiles per super-tile (T = 32)
 constexpr uint32_t kOffCoords = kOffBars + 512;                    // 2 groups x 2 x kMaxPack TileCoords
-constexpr uint32_t kOffBlocks = kOffCoords + 2 * 2 * kMaxPack * 32;
+constexpr uint32_t kCoordBytes = 48;
+constexpr uint32_t kOffBlocks = kOffCoords + 2 * 2 * kMaxPack * kCoordBytes;
 constexpr uint32_t kSmemBytes = kOffBlocks + kMaxSmemBlocks * 24 + 1024;   // + alignment slack
+constexpr float kTinyNorm = 1.0f / 1024.0f;   // below this normalised norm a tile keeps bf16 operands
 
 struct TileCoord {
   int32_t blk;       // -1: no tile
   int32_t x0, y0, cols;
+  int32_t h, w;      // the tile's extent (edge tiles smaller)
   int32_t tm[kNumRoles];
+  int32_t pad[2];
 };
 
 // What the tile decoder needs of a DevBlock, kept in shared memory (used when
@@ -87,24 +101,29 @@ struct SBlock {
   int32_t cols;
   uint16_t tiles_c, T;
   int16_t tm[kNumRoles];
-  int32_t pad;
+  int32_t rows;
 };
 static_assert(sizeof(SBlock) == 24, "SBlock layout");
-static_assert(sizeof(TileCoord) == 32, "TileCoord layout");
+static_assert(sizeof(TileCoord) == kCoordBytes, "TileCoord layout");
 
 struct Smem {
   uint8_t *base;
   __device__ uint8_t *x(int g) const { return base + g * kGroupBytes + kOffX; }
   __device__ uint8_t *s(int g) const { return base + g * kGroupBytes + kOffS; }
   __device__ uint8_t *w(int g) const { return base + g * kGroupBytes + kOffW; }
-  __device__ uint64_t *bar(int g, int i) const { return reinterpret_cast<uint64_t *>(base + kOffBars) + 4 * g + i; }
+  __device__ uint64_t *bar(int g, int i) const { return reinterpret_cast<uint64_t *>(base + kOffBars) + 8 * g + i; }
   __device__ uint64_t *bar_ld(int g) const { return bar(g, 0); }    // M (or input) and G landed
   __device__ uint64_t *bar_w(int g) const { return bar(g, 1); }     // W landed
   __device__ uint64_t *bar_mma(int g) const { return bar(g, 2); }   // the group's MMA job finished
   __device__ uint64_t *bar_never(int g) const { return bar(g, 3); } // never arrived on (stall self-test)
-  __device__ float *red(int g) const { return reinterpret_cast<float *>(base + kOffBars + 64) + kGroupWarps * g; }
-  __device__ uint32_t *tmem_slot() const { return reinterpret_cast<uint32_t *>(base + kOffBars + 128); }
-  __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(base + kOffBars + 132); }
+  __device__ uint64_t *bar_ready(int g) const { return bar(g, 4); } // the operands of the group's next job are written
+  __device__ uint64_t *bar_pro(int g) const { return bar(g, 5); }   // prologue: M' and the partial norms written
+  __device__ uint64_t *bar_epi(int g) const { return bar(g, 6); }   // epilogue: W' / O staged for the stores
+  __device__ float *red(int g) const { return reinterpret_cast<float *>(base + kOffBars + 128) + kGroupWarps * g; }
+  __device__ uint32_t *tmem_slot() const { return reinterpret_cast<uint32_t *>(base + kOffBars + 192); }
+  __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(base + kOffBars + 196); }
+  // operand type of the group's current super-tile (1: fp16), for the issuer
+  __device__ volatile int *fmt16(int g) const { return reinterpret_cast<volatile int *>(base + kOffBars + 200) + g; }
   __device__ SBlock *blocks() const { return reinterpret_cast<SBlock *>(base + kOffBlocks); }
   // current (i = 0) / next (i = 1) super-tile's tile coordinates of group g,
   // kMaxPack each (read and written by the group's issuing thread only)
@@ -236,7 +255,8 @@ __device__ __forceinline__ bool use_smem_blocks(const ResidentArgs &a) {
 __device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, const Smem &sm, int64_t tile, int hint = -1) {
   TileCoord t;
   t.blk = -1;
-  t.x0 = t.y0 = t.cols = 0;
+  t.x0 = t.y0 = t.cols = t.h = t.w = 0;
+  t.pad[0] = t.pad[1] = 0;
 #pragma unroll
   for (int r = 0; r < kNumRoles; ++r) t.tm[r] = -1;
   if (tile >= a.n_tiles) return t;
@@ -258,6 +278,8 @@ __device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, const Sm
     t.y0 = (local / b.tiles_c) * b.T;
     t.x0 = (local % b.tiles_c) * b.T;
     t.cols = b.cols;
+    t.h = min(static_cast<int32_t>(b.T), b.rows - t.y0);
+    t.w = min(static_cast<int32_t>(b.T), b.cols - t.x0);
 #pragma unroll
     for (int r = 0; r < kNumRoles; ++r) t.tm[r] = b.tm[r];
     return t;
@@ -272,6 +294,8 @@ __device__ __forceinline__ TileCoord decode_tile(const ResidentArgs &a, const Sm
   t.y0 = static_cast<int32_t>(local / b.tiles_c) * b.T;
   t.x0 = static_cast<int32_t>(local % b.tiles_c) * b.T;
   t.cols = b.cols;
+  t.h = min(b.T, b.rows - t.y0);
+  t.w = min(b.T, b.cols - t.x0);
 #pragma unroll
   for (int r = 0; r < kNumRoles; ++r) t.tm[r] = b.tmap[r];
   return t;
@@ -370,46 +394,48 @@ enum Job { kJobGram = 0, kJobSquare = 1, kJobUpdate = 2 };
 
 // All threads of the group have written (and fenced) the operands of `job`:
 // one thread issues its eight 128x128x16 MMAs and commits them to bar_mma.
-template <int F, int JOB>
-__device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st);
+// f16: the operands are fp16 (else bf16).
+template <int JOB>
+__device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st, bool f16);
 
-// The barrier also ORs the threads' failure flags: if any thread of the group
-// saw a wait give up, nothing is issued and every thread learns to stop
-// (returns true), at the same point.
-template <int F, int JOB>
-__device__ __forceinline__ bool group_issue(const ResidentArgs &a, const Smem &sm, int g, int gt, uint32_t dP,
-                                            const ResidentStep *st, bool bad) {
-  if (named_bar_or(1 + g, kGroupThreads, bad)) return true;
-  if (gt >= 32) return false;
-  // Lanes 1..31 of the issuing warp wait here for lane 0: if they went on to
-  // spin on the completion barrier, the warp would interleave their
-  // (suspending) try_wait with lane 0's issue and delay the MMAs.
-  if (gt == 0) group_issue_mmas<F, JOB>(sm, g, dP, st);
+// A warp of group g has written (and fenced) its share of the operands of
+// the group's next job: its lane 0 arrives on the group's ready barrier, which
+// completes once all eight warps have arrived; the issuer warp then issues.
+__device__ __forceinline__ void group_ready(const Smem &sm, int g, int lane) {
   __syncwarp();
-  return false;
+  if (lane == 0) mbar_arrive(sm.bar_ready(g));
 }
 
-template <int F, int JOB>
-__device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st) {
+// Bounded group-wide barrier on an mbarrier of count kGroupWarps (one arrival
+// per warp); unlike a named barrier it never hangs a thread whose partners
+// have stopped after a failure.
+__device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t parity, const Smem &sm, int lane, int *status) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  return wait_or_abort(bar, parity, sm, status);
+}
+
+template <int JOB>
+__device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st, bool f16) {
   tc_fence_after();
   const uint64_t tk = sw128_desc(0, 16, 1024);
   const uint32_t dX = dP + 128u;
   // packed A operand: K columns 0..63 at region + [0, 32), 64..127 at region + [64, 96)
   if (JOB == kJobGram) {
     const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
-    constexpr uint32_t id = idesc_f16(128, 128, F, 0, 0, 0);
+    const uint32_t id = f16 ? idesc_f16(128, 128, 0, 0, 0, 0) : idesc_f16(128, 128, 1, 0, 0, 0);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) mma_ts(dP, dX + (kk >> 2) * 64 + (kk & 3) * 8, desc_k(tk, x4, kk), id, kk > 0);
   } else if (JOB == kJobSquare) {
     const uint32_t s4 = smem_u32(sm.s(g)) >> 4;
-    const uint32_t id = idesc_f16(128, 128, F, 0, 0, st->neg2);
+    const uint32_t id = idesc_f16(128, 128, f16 ? 0 : 1, 0, 0, st->neg2);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
       mma_ts(dP, dX + (kk >> 2) * 64 + (kk & 3) * 8, desc_k(tk, s4, kk), id, st->acc2 | (kk > 0));
   } else {
     const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
     const uint64_t tmn = sw128_desc(0, kHalf, 1024);
-    constexpr uint32_t id = idesc_f16(128, 128, F, 0, 1, 0);
+    const uint32_t id = f16 ? idesc_f16(128, 128, 0, 0, 1, 0) : idesc_f16(128, 128, 1, 0, 1, 0);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) mma_ts(dX, dP + (kk >> 2) * 64 + (kk & 3) * 8, desc_mn(tmn, x4, kk), id, kk > 0);
   }
@@ -418,7 +444,14 @@ __device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t
 
 // ------------------------------------------------------------------ one tile group
 // P tiles of edge T = 128 / P per super-tile (P = 1: one 128-tile).
-template <int F, int P>
+//
+// Synchronisation inside a group uses only mbarriers with bounded waits (no
+// named barriers), so a thread whose partners stopped after a failure never
+// hangs: every wait gives up after kWaitLimitNs or as soon as the CTA's abort
+// flag is raised.  Warps agree on a failure among their lanes (a warp stops as
+// a whole); warps of a group that are still running then stop at their next
+// wait, which the abort flag ends.
+template <int P>
 __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem, int g) {
   constexpr uint32_t T = 128 / P;
   const int gt = threadIdx.x - g * kGroupThreads;
@@ -433,22 +466,22 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
   const uint32_t tP = dP + ((q * 32) << 16);           // this warp's lanes of D_P
   const uint32_t tX = tP + 128u;                       // ... and of D_X
   uint8_t *Xs = sm.x(g), *Ss = sm.s(g), *Ws = sm.w(g);
-  const int bar_id = 1 + g;
   const bool step_mode = a.mode == 1;
   const bool has_w = step_mode && a.has_w;
   const int64_t grid = gridDim.x;
   const int64_t n_super = (a.n_tiles + P - 1) / P;
   uint32_t it = 0, job = 0;
   bool mg_issued = false;   // (issuing thread) this super-tile's M/G loads went out during the previous one
-  // (issuing thread) phases armed on / waited for on bar_ld, bar_w and bar_mma,
-  // so that an aborted tile can wait for its own copies and MMAs in flight
-  uint32_t ld_armed = 0, ld_seen = 0, w_armed = 0, w_seen = 0, mma_armed = 0, mma_seen = 0;
+  // (issuing thread) phases armed on / waited for on bar_ld and bar_w, so
+  // that an aborted tile can wait for its own copies in flight
+  uint32_t ld_armed = 0, ld_seen = 0, w_armed = 0, w_seen = 0;
   // Self-test of the timeout path: one group waits on a barrier that nothing
   // arrives on, times out, records HIMUON_ERR_TIMEOUT and makes the CTA abort.
   if (a.test_stall && blockIdx.x == 0 && g == 0) wait_or_abort(sm.bar_never(g), 0, sm, a.status);
   const bool stalled = *sm.abort_flag() != 0;
   TileCoord *cur = sm.coord(g, 0), *nxt = sm.coord(g, 1);
   if (gt == 0) decode_super<P>(a, sm, blockIdx.x + g * grid, cur);
+  __syncwarp();
 
   for (int64_t st = blockIdx.x + g * grid; st < n_super && !stalled; st += 2 * grid, ++it) {
     // this row's tile exists (the last super-tile may hold fewer than P tiles)
@@ -465,10 +498,9 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       }
     }
     __syncwarp();
-    // A failed wait is only recorded here; the group stops together at its
-    // next barrier (a thread leaving alone would strand the others there).
     bool bad = !wait_or_abort(sm.bar_ld(g), it & 1u, sm, a.status);
-    if (!bad) ++ld_seen;
+    if (gt == 0 && !bad) ++ld_seen;
+    if (__any_sync(0xffffffffu, bad)) break;
 
     // ---- prologue: M' = mu M + G (or the plain input), ||.||_F, fp32 copy to D_X.
     // M' (bf16, for the write-back) replaces G in S_s, so X_s is free for X_0 at once.
@@ -506,8 +538,11 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     sumsq = warp_sum(sumsq);
     if (lane == 0) sm.red(g)[wig] = sumsq;
     if (step_mode) fence_proxy_async_smem();
+    tc_fence_before();
     // M' complete in S_s, partial sums visible, M read
-    if (named_bar_or(bar_id, kGroupThreads, bad)) break;
+    bad = !group_sync(sm.bar_pro(g), it & 1u, sm, lane, a.status);
+    if (__any_sync(0xffffffffu, bad)) break;
+    tc_fence_after();
     if (step_mode && gt == 0) {
 #pragma unroll
       for (int j = 0; j < P; ++j)
@@ -515,22 +550,39 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       bulk_commit();
     }
     __syncwarp();
-    float total = 0.f;   // ||tile||^2 of this row's tile: the warps whose rows lie in it
+    // ||tile||^2 of every tile of the super-tile (the warps whose rows lie in it)
+    float tot[P];
 #pragma unroll
-    for (int w = 0; w < kGroupWarps; ++w)
-      if (P == 1 || (32u * (w & 3)) / T == jr) total += sm.red(g)[w];
+    for (int j = 0; j < P; ++j) tot[j] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kGroupWarps; ++w) tot[(32u * (w & 3)) / T] += sm.red(g)[w];
+    float total = tot[0];   // this row's tile (a select, not an indexed load)
+#pragma unroll
+    for (int j = 1; j < P; ++j) total = (jr == static_cast<uint32_t>(j)) ? tot[j] : total;
     const float rho = (sqrtf(total) + a.eps) * a.safety;
+    // operand type of this super-tile (the same in every thread of the group)
+    bool f16 = a.op_fmt == 0;
+    if (!f16 && a.f16_small) {
+      bool small = true;
+      if (P == 1) small = min(cur[0].h, cur[0].w) <= 64;
+      bool tiny = false;
+#pragma unroll
+      for (int j = 0; j < P; ++j) {
+        const float nrm = sqrtf(tot[j]);
+        tiny = tiny || (tot[j] > 0.f && nrm < kTinyNorm * ((nrm + a.eps) * a.safety));
+      }
+      f16 = small && !tiny;
+    }
+    if (gt == 0) *sm.fmt16(g) = f16 ? 1 : 0;   // read by the issuer after this group's next arrival
 
     // ---- operand g_0 X_0 = r(g_0 M' / rho) to X_s and (packed) to D_X
-    tmem_row_to_op<F, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
-    // M' must have left S_s before the first conversion overwrites it; that
-    // conversion follows MMA1, which the issuing thread starts only after this.
+    if (f16) tmem_row_to_op<0, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
+    else tmem_row_to_op<1, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
+    // M' must have left S_s before the first conversion (after MMA1) overwrites it
     if (step_mode && gt == 0) bulk_wait_read0();
-    __syncwarp();
     fence_proxy_async_smem();
     tc_fence_before();
-    if (group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr, bad)) break;
-    ++mma_armed;
+    group_ready(sm, g, lane);
 
     if (gt == 0) {   // next super-tile of this group, while MMA1 runs
       decode_super<P>(a, sm, st + 2 * grid, nxt);
@@ -549,40 +601,48 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       const ResidentStep *stp = &a.step[t];
       // after MMA1: S = r(s D_P) (s = 1 unless c = 0) to S_s and (packed) to D_X
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
-      if (!bad) ++mma_seen;
+      if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
-      if (stp->s == 1.f) tmem_row_to_op<F, false>(tP, tX, Ss, r, hf, 1.f);
-      else tmem_row_to_op<F, true>(tP, tX, Ss, r, hf, stp->s);
+      if (f16) {
+        if (stp->s == 1.f) tmem_row_to_op<0, false>(tP, tX, Ss, r, hf, 1.f);
+        else tmem_row_to_op<0, true>(tP, tX, Ss, r, hf, stp->s);
+      } else {
+        if (stp->s == 1.f) tmem_row_to_op<1, false>(tP, tX, Ss, r, hf, 1.f);
+        else tmem_row_to_op<1, true>(tP, tX, Ss, r, hf, stp->s);
+      }
       fence_proxy_async_smem();
       tc_fence_before();
-      if ((stop = group_issue<F, kJobSquare>(a, sm, g, gt, dP, stp, bad))) break;
-      ++mma_armed;
+      group_ready(sm, g, lane);
       // after MMA2: Bop = r(beta D_P + a I) (beta = b / g^2), packed in D_P
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
-      if (!bad) ++mma_seen;
+      if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
-      tmem_row_to_tmem_op<F>(tP, r, hf, stp->beta, stp->a);
+      if (f16) tmem_row_to_tmem_op<0>(tP, r, hf, stp->beta, stp->a);
+      else tmem_row_to_tmem_op<1>(tP, r, hf, stp->beta, stp->a);
       tc_fence_before();
-      if ((stop = group_issue<F, kJobUpdate>(a, sm, g, gt, dP, stp, bad))) break;
-      ++mma_armed;
+      group_ready(sm, g, lane);
       // after MMA3: next operand r(xr D_X) = g_{t+1} X_{t+1} (xr = 1 for constant coefficients)
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
-      if (!bad) ++mma_seen;
+      if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
       if (t + 1 < a.K) {
-        if (stp->xr == 1.f) tmem_row_to_op<F, false>(tX, tX, Xs, r, hf, 1.f);
-        else tmem_row_to_op<F, true>(tX, tX, Xs, r, hf, stp->xr);
+        if (f16) {
+          if (stp->xr == 1.f) tmem_row_to_op<0, false>(tX, tX, Xs, r, hf, 1.f);
+          else tmem_row_to_op<0, true>(tX, tX, Xs, r, hf, stp->xr);
+        } else {
+          if (stp->xr == 1.f) tmem_row_to_op<1, false>(tX, tX, Xs, r, hf, 1.f);
+          else tmem_row_to_op<1, true>(tX, tX, Xs, r, hf, stp->xr);
+        }
         fence_proxy_async_smem();
         tc_fence_before();
-        if ((stop = group_issue<F, kJobGram>(a, sm, g, gt, dP, nullptr, bad))) break;
-        ++mma_armed;
+        group_ready(sm, g, lane);
       }
     }
     if (stop) break;
 
     // X_s is free now (and S_s unless it stages O): start the next super-tile's loads
     mg_issued = false;
-    if (gt == 0 && nxt[0].blk >= 0 && !a.has_o && !bad) {
+    if (gt == 0 && nxt[0].blk >= 0 && (!step_mode || !a.has_o)) {
       issue_mg<P>(a, sm, g, nxt);
       ++ld_armed;
       mg_issued = true;
@@ -591,9 +651,9 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
 
     // ---- epilogue: O = D_X;  W <- W - lr O  (this row's diagonal block only)
     if (has_w) {
-      const bool wbad = !wait_or_abort(sm.bar_w(g), it & 1u, sm, a.status);
-      if (!wbad) ++w_seen;
-      bad = bad || wbad;
+      bad = !wait_or_abort(sm.bar_w(g), it & 1u, sm, a.status);
+      if (gt == 0 && !bad) ++w_seen;
+      if (__any_sync(0xffffffffu, bad)) break;
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -608,10 +668,10 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
           const uint32_t off = stage_off<P>(jr, rr, cg - jr * (T / 8));
           const float *o = v + 8 * k;   // gamma_{K-1} O
           if (a.has_o) {
-            float os[8];
+            float ov[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) os[e] = a.oscale * o[e];
-            *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(os);
+            for (int e = 0; e < 8; ++e) ov[e] = a.oscale * o[e];
+            *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(ov);
           }
           if (has_w) {
             const float lro = -a.lr * a.oscale;
@@ -626,32 +686,107 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    if (named_bar_or(bar_id, kGroupThreads, bad)) break;
+    // Only the storing thread needs the whole group's W' / O in place; the
+    // others go on to the next super-tile, whose loads wait for these stores.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.bar_epi(g));
     if (gt == 0) {
+      bad = !wait_or_abort(sm.bar_epi(g), it & 1u, sm, a.status);
+      if (!bad) {
 #pragma unroll
-      for (int j = 0; j < P; ++j) {
-        if (cur[j].blk < 0) continue;
-        if (a.has_o) store_tile<P>(a.tmaps + cur[j].tm[kRoleOut], Ss, cur[j], j);
-        if (has_w) store_tile<P>(a.tmaps + cur[j].tm[kRoleW], Ws, cur[j], j);
+        for (int j = 0; j < P; ++j) {
+          if (cur[j].blk < 0) continue;
+          if (a.has_o) store_tile<P>(a.tmaps + cur[j].tm[kRoleOut], Ss, cur[j], j);
+          if (has_w) store_tile<P>(a.tmaps + cur[j].tm[kRoleW], Ws, cur[j], j);
+        }
+        bulk_commit();
       }
-      bulk_commit();
 #pragma unroll
       for (int j = 0; j < P; ++j) cur[j] = nxt[j];
     }
-    __syncwarp();
+    if (__any_sync(0xffffffffu, bad)) break;
   }
   if (gt == 0) {
-    // After an abort: wait (bounded) for this group's own loads and MMAs still
-    // in flight, so that no copy lands in, and no MMA touches, memory the CTA
-    // is about to release.  Nothing is outstanding after a normal finish.
+    // After an abort: wait (bounded) for this group's own loads still in
+    // flight, so that no copy lands in memory the CTA is about to release
+    // (the issuer waits for the group's MMAs).  Nothing is outstanding after a
+    // normal finish.
     for (; ld_seen < ld_armed; ++ld_seen) mbar_wait(sm.bar_ld(g), ld_seen & 1u, a.status);
     for (; w_seen < w_armed; ++w_seen) mbar_wait(sm.bar_w(g), w_seen & 1u, a.status);
-    for (; mma_seen < mma_armed; ++mma_seen) mbar_wait(sm.bar_mma(g), mma_seen & 1u, a.status);
     bulk_wait0();
   }
 }
 
-template <int F, int P>
+// ------------------------------------------------------------------ the issuer
+// One thread (lane 0 of warp 16) issues every MMA of both groups: it polls
+// each group's ready barrier (non-blocking) and, when a group's operands are
+// in place, issues that group's next job and commits it to the group's MMA
+// barrier.  The converting warps therefore never stall in an MMA issue while
+// the tensor pipe is busy with the other group's job.  Per group it walks the
+// same sequence as the group: per super-tile K steps of (Gram, Square, Update).
+template <int P>
+__device__ void issuer_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem) {
+  const int64_t grid = gridDim.x;
+  const int64_t n_super = (a.n_tiles + P - 1) / P;
+  int64_t st0 = blockIdx.x, st1 = blockIdx.x + grid;
+  int t0 = 0, t1 = 0, jb0 = kJobGram, jb1 = kJobGram;
+  uint32_t rph0 = 0, rph1 = 0, issued0 = 0, issued1 = 0;
+  bool done0 = st0 >= n_super, done1 = st1 >= n_super;
+  uint64_t last = globaltimer_ns();
+  uint32_t spin = 0;
+  while (!(done0 && done1)) {
+    bool any = false;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      // this group's state (named per group: no local-memory arrays)
+      int64_t &st = g == 0 ? st0 : st1;
+      int &t = g == 0 ? t0 : t1;
+      int &jb = g == 0 ? jb0 : jb1;
+      uint32_t &rph = g == 0 ? rph0 : rph1;
+      uint32_t &issued = g == 0 ? issued0 : issued1;
+      bool &done = g == 0 ? done0 : done1;
+      if (done) continue;
+      if (!mbar_test_wait(sm.bar_ready(g), rph & 1u)) continue;
+      ++rph;
+      tc_fence_after();
+      const bool f16 = *sm.fmt16(g) != 0;
+      const uint32_t dP = tmem + 256u * g;
+      const ResidentStep *stp = &a.step[t];
+      if (jb == kJobGram) group_issue_mmas<kJobGram>(sm, g, dP, nullptr, f16);
+      else if (jb == kJobSquare) group_issue_mmas<kJobSquare>(sm, g, dP, stp, f16);
+      else group_issue_mmas<kJobUpdate>(sm, g, dP, stp, f16);
+      ++issued;
+      // next job of this group: the Gram job of step t + 1, or of the next super-tile
+      if (++jb == 3) {
+        jb = kJobGram;
+        if (++t == a.K) {
+          t = 0;
+          st += 2 * grid;
+          done = st >= n_super;
+        }
+      }
+      any = true;
+    }
+    if (any) {
+      last = globaltimer_ns();
+      spin = 0;
+    } else if ((++spin & 63u) == 0) {
+      if (*sm.abort_flag()) break;
+      if (globaltimer_ns() - last > kWaitLimitNs) {
+        set_status(a.status, HIMUON_ERR_TIMEOUT);
+        *sm.abort_flag() = 1;
+        break;
+      }
+    }
+  }
+  // Every MMA issued must have finished before the CTA frees its TMEM and
+  // shared memory: wait (bounded) for each group's last job.  Jobs of a group
+  // complete in order, one barrier phase each.
+  if (issued0 > 0) mbar_wait(sm.bar_mma(0), (issued0 - 1u) & 1u, a.status);
+  if (issued1 > 0) mbar_wait(sm.bar_mma(1), (issued1 - 1u) & 1u, a.status);
+}
+
+template <int P>
 __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_constant__ ResidentArgs args) {
   extern __shared__ uint8_t smem_raw[];
   Smem sm;
@@ -663,6 +798,10 @@ __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_c
       mbar_init(sm.bar_w(g), 1);
       mbar_init(sm.bar_mma(g), 1);
       mbar_init(sm.bar_never(g), 1);
+      mbar_init(sm.bar_ready(g), kGroupWarps);
+      mbar_init(sm.bar_pro(g), kGroupWarps);
+      mbar_init(sm.bar_epi(g), kGroupWarps);
+      *sm.fmt16(g) = 0;
     }
     *sm.abort_flag() = 0;
     fence_mbar_init();
@@ -681,7 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_c
       d.T = static_cast<uint16_t>(b.T);
 #pragma unroll
       for (int r = 0; r < kNumRoles; ++r) d.tm[r] = static_cast<int16_t>(b.tmap[r]);
-      d.pad = 0;
+      d.rows = b.rows;
     }
   }
   tc_fence_before();
@@ -689,7 +828,12 @@ __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_slot();
 
-  group_main<F, P>(args, sm, tmem, warp / kGroupWarps);
+  if (warp < kIssuerWarp) {
+    group_main<P>(args, sm, tmem, warp / kGroupWarps);
+  } else {
+    if ((threadIdx.x & 31) == 0) issuer_main<P>(args, sm, tmem);
+    __syncwarp();
+  }
 
   tc_fence_before();
   __syncthreads();
@@ -701,6 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_resident_kernel(const __grid_c
 }
 
 }  // namespace
+
 
 int resident_smem_bytes() { return static_cast<int>(kSmemBytes); }
 int resident_max_smem_blocks() { return kMaxSmemBlocks; }
@@ -740,23 +885,22 @@ void make_resident_steps(ResidentArgs &args, const float *coeffs, int K) {
   args.oscale = K > 0 ? static_cast<float>(1.0 / gam[K - 1]) : 1.f;
 }
 
-template <int F, int P>
-static cudaError_t launch_fmt(const ResidentArgs &args, int grid, cudaStream_t stream) {
+template <int P>
+static cudaError_t launch_pack(const ResidentArgs &args, int grid, cudaStream_t stream) {
   // The shared-memory opt-in is per device; setting it again is cheap.
-  cudaError_t e = cudaFuncSetAttribute(ns_resident_kernel<F, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(ns_resident_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   count_launch();
-  ns_resident_kernel<F, P><<<grid, kThreads, kSmemBytes, stream>>>(args);
+  ns_resident_kernel<P><<<grid, kThreads, kSmemBytes, stream>>>(args);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ns_resident(const ResidentArgs &args, int grid, cudaStream_t stream) {
-  const bool f16 = args.op_fmt == 0;
   switch (args.pack) {
-    case 2: return f16 ? launch_fmt<0, 2>(args, grid, stream) : launch_fmt<1, 2>(args, grid, stream);
-    case 4: return f16 ? launch_fmt<0, 4>(args, grid, stream) : launch_fmt<1, 4>(args, grid, stream);
-    default: return f16 ? launch_fmt<0, 1>(args, grid, stream) : launch_fmt<1, 1>(args, grid, stream);
+    case 2: return launch_pack<2>(args, grid, stream);
+    case 4: return launch_pack<4>(args, grid, stream);
+    default: return launch_pack<1>(args, grid, stream);
   }
 }
 

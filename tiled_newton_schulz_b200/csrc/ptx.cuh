@@ -56,6 +56,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test: has the phase with parity `phase` completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait for the phase with parity `phase` to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, int *status) {
   if (mbar_try_wait(bar, phase)) return true;

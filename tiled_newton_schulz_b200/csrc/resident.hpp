@@ -31,6 +31,7 @@ struct ResidentArgs {
   int32_t mode;     // 0: NS in -> out; 1: momentum step
   int32_t has_w, has_o;
   int32_t op_fmt;   // tensor-core operand type: 0 fp16, 1 bf16
+  int32_t f16_small;  // bf16 call: super-tiles of tiles with short side <= 64 use fp16 operands
   int32_t smem_blocks;  // 1: the block table fits the kernel's compact shared-memory copy
   int32_t pack;     // tiles per 128 x 128 super-tile: 1 (T = 128), 2 (T = 64) or 4 (T = 32)
   int32_t test_stall;  // self-test: CTA 0 waits on a barrier nothing arrives on (timeout path)

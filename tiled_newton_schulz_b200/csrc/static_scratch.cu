@@ -9,6 +9,8 @@
 // cudaGetSymbolAddress, looked up once per device with that device current.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "himuon.h"
 
 namespace himuon {
@@ -21,7 +23,10 @@ namespace {
 __device__ __align__(256) unsigned char g_static_scratch[HIMUON_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices] = {};
+// Looked-up addresses, one per device.  Host threads may race on a device's
+// first call: each then looks the address up itself (the same value) and the
+// atomic store keeps the slot well defined.
+std::atomic<void *> g_scratch_addr[kMaxDevices];
 
 // Device address of g_static_scratch on the current device (set-up on first use).
 int scratch_address(void **out) {
@@ -31,16 +36,16 @@ int scratch_address(void **out) {
     return HIMUON_ERR_NO_DEVICE;
   }
   if (dev < 0 || dev >= kMaxDevices) return HIMUON_ERR_NO_DEVICE;
-  if (!g_scratch_addr[dev]) {
-    void *ptr = nullptr;
+  void *ptr = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!ptr) {
     const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
     if (e != cudaSuccess || !ptr) {
       cudaGetLastError();
       return HIMUON_ERR_CUDA;
     }
-    g_scratch_addr[dev] = ptr;
+    g_scratch_addr[dev].store(ptr, std::memory_order_release);
   }
-  *out = g_scratch_addr[dev];
+  *out = ptr;
   return HIMUON_OK;
 }
 
