@@ -11,9 +11,17 @@ O = tiledNS_T(M) with K = 5 quintic steps, W <- W - 0.02 O, all bf16 in HBM
 
 A step is one himuon_momentum_step call over all matrices.  The inputs
 (38.9 GB) are far larger than L2 (126 MB), so no flush is needed between
-steps.  Time is taken with CUDA events on the launching stream; with N > 1
-every rank runs its own replica of the workload (the tiles are independent:
-no data-path collective) and the max over ranks is reported.
+steps.  Time is taken with CUDA events on the launching stream.
+
+With N > 1 (under torchrun, one rank per GPU, NCCL) the step is the
+data-parallel sharded step of ``shard.flat_sharded_step``: every rank holds
+the replicated weights and its own gradients for the whole 7B set in flat
+buffers, the gradients are reduce-scattered (averaged) onto the owners of the
+matrices, each rank runs the fused library step on its own matrices (the
+momentum lives only there), and the weights are all-gathered, in buckets that
+overlap the collectives with the steps.  The job processes the 7B set once
+per step (strong scaling); the max over ranks is reported.  ``--sharded``
+runs the same code path on one rank.
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on the host cores.
@@ -219,19 +227,114 @@ def run_reference(args):
     return 0
 
 
+def run_sharded(args):
+    """The data-parallel sharded step (N ranks, NCCL) on the 7B set."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from tiled_newton_schulz_b200 import himuon as hm
+    from tiled_newton_schulz_b200 import shard
+    from tiled_newton_schulz_b200.inputs import gaussian_torch, low_rank_plus_noise_torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world == 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29511")
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    hm.load()
+    T = args.tile
+    compute = {"bf16": hm.BF16, "fp16": hm.FP16}[args.compute]
+    mats = llama7b_matrices(args.layers)
+    shapes, splits = [s for s, _ in mats], [sp for _, sp in mats]
+    elements = sum(H * Wd for H, Wd in shapes)
+    n_tiles, flops = workload_tiles(mats, T)
+    fs = shard.FlatShards(shapes, splits, T, world, buckets=args.buckets)
+    W_flat = torch.empty(fs.total, dtype=torch.bfloat16, device=device)
+    G_flat = torch.empty_like(W_flat)
+    M_mine = torch.empty(fs.mine_total, dtype=torch.bfloat16, device=device)
+    Wv, Gv, Mv = fs.views(W_flat), fs.views(G_flat), fs.mine_views(M_mine, rank)
+    for i, (H, Wd) in enumerate(shapes):
+        # the same weights on every rank, this rank's own gradients, momentum on the owner
+        Wv[i].copy_(gaussian_torch(H, Wd, 3 * i, device, torch.float32) * 0.02)
+        Gv[i].copy_(low_rank_plus_noise_torch(H, Wd, 64, 0.01, 1000 * rank + 3 * i + 2, device))
+        if Mv[i] is not None:
+            Mv[i].copy_(low_rank_plus_noise_torch(H, Wd, 64, 0.01, 3 * i + 1, device))
+    torch.cuda.synchronize(device)
+    p = hm.params(T, QUINTIC, steps=K_STEPS, compute=compute)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        shard.flat_sharded_step(W_flat, G_flat, M_mine, fs, MU, LR, p)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    st = hm.device_status()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.4)
+    dist.barrier()
+    torch.cuda.synchronize(device)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    launches0 = hm.launch_count()
+    evs[0].record(stream)
+    for i in range(args.steps):
+        step()
+        evs[i + 1].record(stream)
+    launches = hm.launch_count() - launches0
+    torch.cuda.synchronize(device)
+    dist.barrier()
+    clk = clocks.stop()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    t = torch.tensor([evs[0].elapsed_time(evs[-1])] + per + [float(st != 0)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, per, bad = float(t[0].item()), [float(v) for v in t[1:-1].tolist()], t[-1].item() > 0
+    ms_step = ms / args.steps
+    peaks, peak_src = read_peaks()
+    peak_burst = float(peaks.get("bf16_tflops"))
+    achieved = flops / (ms_step / 1e3) / 1e12
+    bytes_coll = 2 * 2.0 * elements * (world - 1) / world   # bf16 reduce-scatter of G + all-gather of W, per rank
+    line = {
+        "metric": METRIC, "value": elements / (ms_step / 1e3), "unit": "elements/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": args.compute, "data": "synthetic",
+        "config": {"workload": f"llama7b_{args.layers}l_full_step_T{T}", "tile": T, "steps_K": K_STEPS, "mu": MU,
+                   "lr": LR, "matrices": len(mats), "tiles": n_tiles, "elements_total": elements,
+                   "storage": "bf16 W, M, G", "accumulate": "fp32",
+                   "l2": f"inputs {6 * elements / 1e9:.1f} GB >> 126 MB L2, no flush",
+                   "parallelism": (f"dp{world}: gradients reduce-scattered onto matrix owners, fused step on own "
+                                   f"matrices, weights all-gathered (NCCL), {fs.buckets} buckets"),
+                   "flop_imbalance": fs.imbalance(T)},
+        "ms_per_step_median": statistics.median(per), "ms_per_step_min": min(per),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_burst * world, "unit": "TFLOP/s",
+                     "frac": achieved / (peak_burst * world), "traffic": None,
+                     "peak_source": f"bf16_tflops x {world} GPUs ({peak_src})",
+                     "collective_bytes_per_rank": bytes_coll,
+                     "collective_time_ms_at_770GBps": bytes_coll / 770e9 * 1e3},
+        "cpu_baseline": None,
+        "e2e": {"value": None, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+                "note": "not measured for the sharded step: the whole gradient of every rank would cross PCIe"},
+        "gpu_launches": launches, "clocks": clk, "device_status_ok": not bad,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
 def run_ours(args):
     import numpy as np
     import torch
     import torch.distributed as dist
     from tiled_newton_schulz_b200 import himuon as hm
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    # one GPU (N > 1 runs the sharded step, run_sharded)
+    world, rank, local = 1, 0, int(os.environ.get("LOCAL_RANK", "0"))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     hm.load()
@@ -274,8 +377,6 @@ def run_ours(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.4)
-    if world > 1:
-        dist.barrier()
     torch.cuda.synchronize(device)
     # one event between consecutive steps: the whole region and every step's time
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
@@ -286,15 +387,9 @@ def run_ours(args):
         evs[i + 1].record(stream)
     launches = hm.launch_count() - launches0
     torch.cuda.synchronize(device)
-    if world > 1:
-        dist.barrier()
     clk = clocks.stop()
     ms = evs[0].elapsed_time(evs[-1])
     per_step_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
-    if world > 1:
-        t = torch.tensor([ms] + per_step_ms, device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, per_step_ms = float(t[0].item()), [float(v) for v in t[1:].tolist()]
     st = hm.device_status()
     if st != 0:
         raise RuntimeError(f"device status after timing: {hm.status_string(st)}")
@@ -356,8 +451,6 @@ def run_ours(args):
 
         e2e_step()
         torch.cuda.synchronize(device)
-        if world > 1:
-            dist.barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         for _ in range(e2e_steps):
@@ -365,10 +458,6 @@ def run_ours(args):
         a1.record(stream)
         torch.cuda.synchronize(device)
         ems = a0.elapsed_time(a1)
-        if world > 1:
-            t = torch.tensor([ems], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
         e2e_value = world * elements / (ems / e2e_steps / 1e3)
         del hW, hM, hG
 
@@ -422,7 +511,7 @@ def run_ours(args):
                    "tiles": n_tiles, "elements_per_gpu": elements, "storage": "bf16 W, M, G",
                    "accumulate": "fp32",
                    "l2": f"inputs {6 * elements / 1e9:.1f} GB per GPU >> 126 MB L2, no flush",
-                   "parallelism": f"replicas x{world} (independent tiles, no collective)"},
+                   "parallelism": "one GPU"},
         "tflops": tflops,
         "ms_per_step_median": statistics.median(per_step_ms), "ms_per_step_min": min(per_step_ms),
         "ms_per_step_max": max(per_step_ms),
@@ -439,11 +528,7 @@ def run_ours(args):
         line["config"].update({"tile_mix": mix, "candidates": list(AUTO_CANDIDATES), "budget_ms": args.budget_ms,
                                "modeled_ms": modeled_ms,
                                "cost_model": "momentum_step per matrix at each T, CUDA events, batched per shape"})
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -476,6 +561,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sharded", action="store_true", help="time the data-parallel sharded step even on one rank")
+    ap.add_argument("--buckets", type=int, default=4, help="buckets of the sharded step's collectives")
     ap.add_argument("--budget-ms", type=float, default=None,
                     help="choose T per matrix at run time: the largest tiles whose measured cost fits this budget")
     args = ap.parse_args()
@@ -483,6 +570,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 or args.sharded:
+        return run_sharded(args)
     return run_ours(args)
 
 

@@ -171,3 +171,95 @@ def test_owners_rejects_bad_assignments():
         shard.owners([[0, 1], [1]], 3)
     with pytest.raises(ValueError):
         shard.owners([[0], [2]], 3)
+
+
+# ---------------------------------------------------------------- flat buffers
+
+def test_flat_placement_is_disjoint_aligned_and_bucketed():
+    wl = inputs.llama7b_set(2)
+    shapes = [(m.rows, m.cols) for m in wl.matrices]
+    splits = [m.split for m in wl.matrices]
+    for world in (1, 2, 3, 8):
+        for buckets in (1, 2, 5):
+            fs = shard.FlatShards(shapes, splits, 128, world, buckets=buckets)
+            spans = sorted((o, o + h * w) for o, (h, w) in zip(fs.offset, shapes))
+            assert all(a % 128 == 0 for a, _ in spans)
+            assert all(b0 <= a1 for (_, b0), (a1, _) in zip(spans, spans[1:]))       # no overlap
+            assert spans[-1][1] <= fs.total
+            for i, (h, w) in enumerate(shapes):
+                r, b = fs.owner[i], fs.bucket_of[i]
+                lo = fs.bucket_base[b] + r * fs.slot_elems[b]
+                assert lo <= fs.offset[i] and fs.offset[i] + h * w <= lo + fs.slot_elems[b]   # inside its slot
+                mo = fs.mine_offset[i]
+                assert 0 <= mo and mo + h * w <= fs.mine_total
+            assert sorted(i for r in range(world) for b in range(fs.buckets) for i in fs.members[r][b]) == \
+                list(range(len(shapes)))
+
+
+def _flat_worker(rank, world, port, q, buckets, broken):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        fs = shard.FlatShards(SHAPES, SPLITS, T, world, buckets=buckets)
+        W0, M0, G0 = _state(rank)
+        W_flat = torch.zeros(fs.total, dtype=torch.float64)
+        G_flat = torch.zeros(fs.total, dtype=torch.float64)
+        M_mine = torch.zeros(fs.mine_total + (1 if broken and rank == 1 else 0), dtype=torch.float64)
+        for v, x in zip(fs.views(W_flat), W0):
+            v.copy_(x)
+        for v, x in zip(fs.views(G_flat), G0):
+            v.copy_(x)
+        for i, v in enumerate(fs.mine_views(M_mine, rank)):
+            if v is not None:
+                v.copy_(M0[i])
+        try:
+            shard.flat_sharded_step(W_flat, G_flat, M_mine, fs, MU, LR, None, step_fn=_oracle_step(T))
+        except ValueError as e:
+            q.put((rank, "raised", str(e)))
+            return
+        mine = {i: v.numpy().copy() for i, v in enumerate(fs.mine_views(M_mine, rank)) if v is not None}
+        q.put((rank, "done", [v.numpy().copy() for v in fs.views(W_flat)], mine))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run_flat(buckets, broken=False):
+    import oracle
+    oracle.build()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_flat_worker, args=(r, 2, port, q, buckets, broken)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(p.exitcode == 0 for p in procs)
+    return sorted(out, key=lambda r: r[0])
+
+
+@pytest.mark.parametrize("buckets", [1, 3])
+def test_two_rank_flat_sharded_step_matches_single_process(buckets):
+    """Reduce-scatter of the gradients, each rank's step on its own matrices,
+    all-gather of the weights: every rank ends with exactly the weights of a
+    single-process step on the averaged gradients, and each owner with its
+    matrices' new momentum."""
+    import oracle
+    out = _run_flat(buckets)
+    assert [o[1] for o in out] == ["done", "done"]
+    W, M, _ = _state(0)
+    G = [(a + b) / 2 for a, b in zip(_state(0)[2], _state(1)[2])]
+    for i in range(len(SHAPES)):
+        mp_ = oracle.momentum(M[i].numpy(), G[i].numpy(), MU)
+        Wr = W[i].numpy() - LR * oracle.ns_tiled_split(mp_, T, [inputs.QUINTIC] * 5, split=SPLITS[i])
+        for o in out:
+            assert np.array_equal(o[2][i], Wr), i
+        owner = [o for o in out if i in o[3]]
+        assert len(owner) == 1 and np.array_equal(owner[0][3][i], mp_), i
+
+
+def test_flat_sharded_step_with_a_bad_buffer_raises_on_every_rank():
+    out = _run_flat(2, broken=True)
+    assert [o[1] for o in out] == ["raised", "raised"]
+    assert "rank 1" in out[1][2] and "another rank" in out[0][2]
