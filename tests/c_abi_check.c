@@ -21,7 +21,7 @@ int main(void) {
   himuon_ns_params p;
   himuon_mat mats[2];
   int64_t records[5 * 16];
-  int32_t tiles[2] = {128, 256};
+  int32_t tiles[2] = {128, 512};
   int64_t n;
 
   CHECK(himuon_version() == HIMUON_VERSION);
@@ -47,7 +47,7 @@ int main(void) {
   CHECK(records[5 * 11 + 1] == 256 && records[5 * 11 + 2] == 384);   /* last tile: row 256, column 384 */
   CHECK(records[5 * 11 + 3] == 44 && records[5 * 11 + 4] == 116);    /* 300 - 256, 500 - 384 */
 
-  /* on chip at T = 128 needs no workspace; a per-matrix T of 256 does */
+  /* on chip at T = 128 (and 256) needs no workspace; a per-matrix T of 512 does */
   mats[1] = mats[0];
   mats[1].data = storage + 0;
   CHECK(himuon_workspace_size(mats, 1, NULL, &p, HIMUON_OP_NS_TILED) == 0);

@@ -82,7 +82,11 @@ NO_B = (1.5, 0.0, -0.5)
 # polar factor: sixteen quintic steps do not contract, and their bf16 operand
 # roundings add up past the 3e-2 budget (an emulation of exactly the kernel's
 # rounding points gives 5.2% bf16 / 3.1% fp16 per tile for them, 2.3% / 0.5%
-# for this list; the GPU matched the emulation).
+# for this list; the GPU matched the emulation).  This list also multiplies a
+# singular value near zero by about 4e4 (3.4445^5 x 1.5^11), so the noise
+# floor of a low-rank-plus-noise tile ends in the steep middle of the map,
+# where an 8-bit operand rounding moves it by ~0.25 (bf16; fp16 keeps it
+# within 0.05; tests/test_rounding_budget.py): its cases run fp16 operands.
 STEP_LISTS = {
     "K1": [QUINTIC_T],
     "K16": [QUINTIC_T] * 5 + [CUBIC] * 11,
@@ -100,7 +104,8 @@ def test_resident_step_lists(hm, steps, T, compute):
     co = STEP_LISTS[steps]
     x = dev(X, torch.bfloat16)
     y = torch.empty_like(x)
-    hm.ns_tiled([x], [y], hm.params(T, co, compute=hm.BF16 if compute == "bf16" else hm.FP16))
+    code = hm.BF16 if (compute == "bf16" and steps != "K16") else hm.FP16
+    hm.ns_tiled([x], [y], hm.params(T, co, compute=code))
     assert hm.device_status() == 0
     c32 = [tuple(float(np.float32(v)) for v in tri) for tri in co]
     check16(to_np(y), oracle.ns_tiled(to_np(x), T, c32), T)
@@ -234,12 +239,12 @@ def test_momentum_step_resident(hm):
                 assert np.linalg.norm(wg[sl] - W2[sl]) <= bound
 
 
-@pytest.mark.parametrize("T", [32, 64, 128])
+@pytest.mark.parametrize("T", [32, 64, 128, 256])
 def test_integer_coded_reassembly_bitexact(hm, T):
     """Tile t holds c_t P_t (signed permutation with its own shift and signs);
     the output keeps support and signs exactly, so any misplaced, swapped or
     transposed tile fails."""
-    H, W = 512, 384
+    H, W = (512, 384) if T < 256 else (768, 640)
     X = np.zeros((H, W))
     for t, (r0, c0, h, w) in enumerate(oracle.tile_grid(H, W, T)):
         P = inputs.signed_permutation(T, shift=(7 * t) % T, sign_bits=(t * 2654435761) & 0x7FFFFFFF)
@@ -361,3 +366,52 @@ def test_gram_ns_per_step_coefficients(hm, restart, T):
     c32 = [tuple(float(np.float32(v)) for v in tri) for tri in GRAM_STEPS]
     ref = oracle.gram_ns_tiled(to_np(x), T, c32, restart=restart)
     check16(to_np(y), ref, T)
+
+
+# T = 256 on a CTA pair: every 256 x 256 tile is split by rows over two CTAs.
+@pytest.mark.parametrize("compute", ["bf16", "fp16"])
+@pytest.mark.parametrize("H,W", [(512, 768), (600, 520), (256, 256), (100, 70), (700, 300), (1, 300), (130, 1000)])
+def test_pair_tiled_ns(hm, H, W, compute):
+    """Ragged edges in both directions, a tile whose second CTA holds only
+    padding (100 x 70, 130 rows), tall tiles, and thin tiles that take fp16
+    operands in a bf16 call (1 x 300)."""
+    X = inputs.gaussian((H, W), seed=11 * H + W)
+    code = hm.BF16 if compute == "bf16" else hm.FP16
+    xin, y = run_ns(hm, X, 256, code, torch.bfloat16)
+    check16(y, oracle.ns_tiled(xin, 256, C32), 256)
+
+
+@pytest.mark.parametrize("steps", sorted(STEP_LISTS))
+def test_pair_step_lists(hm, steps):
+    X = inputs.low_rank_plus_noise(512, 768, inputs.sigma_inverse(32), 0.01, seed=3 + len(steps))
+    co = STEP_LISTS[steps]
+    x = dev(X, torch.bfloat16)
+    y = torch.empty_like(x)
+    hm.ns_tiled([x], [y], hm.params(256, co, compute=hm.FP16 if steps == "K16" else hm.BF16))
+    assert hm.device_status() == 0
+    c32 = [tuple(float(np.float32(v)) for v in tri) for tri in co]
+    check16(to_np(y), oracle.ns_tiled(to_np(x), 256, c32), 256)
+
+
+def test_pair_momentum_step(hm):
+    """The fused step on the pair kernel: M' within one bf16 ulp, O against
+    the oracle, W' = W - lr O."""
+    shapes = [(512, 512), (300, 700), (768, 256)]
+    rng = np.random.default_rng(21)
+    w = [dev(0.02 * rng.standard_normal(sh), torch.bfloat16) for sh in shapes]
+    m = [dev(inputs.low_rank_plus_noise(*sh, inputs.sigma_inverse(16), 0.01, seed=500 + i), torch.bfloat16)
+         for i, sh in enumerate(shapes)]
+    g = [dev(inputs.low_rank_plus_noise(*sh, inputs.sigma_inverse(16), 0.01, seed=600 + i), torch.bfloat16)
+         for i, sh in enumerate(shapes)]
+    o = [torch.empty_like(x) for x in m]
+    w0, m0, g0 = [to_np(x) for x in w], [to_np(x) for x in m], [to_np(x) for x in g]
+    hm.momentum_step(w, m, g, 0.95, 0.02, hm.params(256, QUINTIC, steps=5), update_out=o)
+    assert hm.device_status() == 0
+    lr32 = float(np.float32(0.02))
+    for i in range(len(shapes)):
+        W2, M2, O = oracle.momentum_step(w0[i], m0[i], g0[i], 0.95, 0.02, 256, C32)
+        assert np.all(np.abs(to_np(m[i]) - M2) <= bf16_ulp(M2))
+        check16(to_np(o[i]), O, 256)
+        got = to_np(o[i])
+        wexp = w0[i] - lr32 * got
+        assert np.all(np.abs(to_np(w[i]) - wexp) <= bf16_ulp(wexp) + lr32 * bf16_ulp(got) + 1e-12)

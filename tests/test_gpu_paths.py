@@ -31,10 +31,13 @@ def dev(x):
     return torch.from_numpy(np.ascontiguousarray(x)).to("cuda", torch.bfloat16)
 
 
-def test_forced_staged_path_agrees_with_on_chip(hm, monkeypatch):
+@pytest.mark.parametrize("T", [128, 256])
+def test_forced_staged_path_agrees_with_on_chip(hm, monkeypatch, T):
+    """The on-chip kernels (T = 128: one CTA per tile group; T = 256: a CTA
+    pair per tile) and the staged GEMMs on the same call."""
     X = inputs.low_rank_plus_noise(384, 512, inputs.sigma_inverse(16), 0.01, seed=21)
     x = dev(X)
-    p = hm.params(128, QUINTIC, steps=5)
+    p = hm.params(T, QUINTIC, steps=5)
     y_chip = torch.empty_like(x)
     hm.ns_tiled([x], [y_chip], p)
     n0 = hm.launch_count()
@@ -45,21 +48,22 @@ def test_forced_staged_path_agrees_with_on_chip(hm, monkeypatch):
     assert hm.launch_count() - n0 > 1          # pack, GEMMs, normalise, unpack: not the one on-chip launch
     monkeypatch.delenv("HIMUON_FORCE_PATH")
     assert hm.device_status() == 0
-    ref = oracle.ns_tiled(to_np(x), 128, C32)
+    ref = oracle.ns_tiled(to_np(x), T, C32)
     a, b = to_np(y_chip), to_np(y_stg)
-    assert per_tile_errors(a, ref, 128).max() <= TOL16
-    assert per_tile_errors(b, ref, 128).max() <= TOL16
-    assert per_tile_errors(a, b, 128).max() <= TOL16
+    assert per_tile_errors(a, ref, T).max() <= TOL16
+    assert per_tile_errors(b, ref, T).max() <= TOL16
+    assert per_tile_errors(a, b, T).max() <= TOL16
 
 
-def test_forced_staged_momentum_step_same_momentum(hm, monkeypatch):
+@pytest.mark.parametrize("T", [128, 256])
+def test_forced_staged_momentum_step_same_momentum(hm, monkeypatch, T):
     """Both paths form M' = mu M + G in fp32 and store it rounded to nearest
     bf16: bit-identical.  W' agrees within the update's tolerance."""
     H, W = 256, 384
     w0 = 0.02 * inputs.gaussian((H, W), seed=1)
     m0 = inputs.low_rank_plus_noise(H, W, inputs.sigma_inverse(16), 0.01, seed=2)
     g0 = inputs.low_rank_plus_noise(H, W, inputs.sigma_inverse(16), 0.01, seed=3)
-    p = hm.params(128, QUINTIC, steps=5)
+    p = hm.params(T, QUINTIC, steps=5)
     out = {}
     for path in ("chip", "staged"):
         if path == "staged":
@@ -70,7 +74,7 @@ def test_forced_staged_momentum_step_same_momentum(hm, monkeypatch):
         out[path] = (to_np(w), to_np(m))
     monkeypatch.delenv("HIMUON_FORCE_PATH")
     assert np.array_equal(out["chip"][1], out["staged"][1])
-    W2, _, O = oracle.momentum_step(to_np(dev(w0)), to_np(dev(m0)), to_np(dev(g0)), 0.95, 0.02, 128, C32)
+    W2, _, O = oracle.momentum_step(to_np(dev(w0)), to_np(dev(m0)), to_np(dev(g0)), 0.95, 0.02, T, C32)
     bound = np.linalg.norm(0.5 * bf16_ulp(W2)) + float(np.float32(0.02)) * TOL16 * np.linalg.norm(O)
     for path in out:
         assert np.linalg.norm(out[path][0] - W2) <= bound

@@ -91,9 +91,13 @@ def test_workspace_size_on_the_host(lib):
     mats = (himuon.Mat * 1)(himuon.Mat(0x1000, 4096, 4096, 4096, himuon.BF16))
     assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p), 0) == 0       # on-chip path
     p256 = himuon.params(256, (3.4445, -4.7750, 2.0315), steps=5)
-    need = lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p256), 0)
-    assert need > 256 * 256 * 8 * 256
-    pc = himuon.params(256, (3.4445, -4.7750, 2.0315), steps=5, chunk_bytes=64 << 20)
+    assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p256), 0) == 0    # on chip, CTA pairs
+    p256f = himuon.params(256, (3.4445, -4.7750, 2.0315), steps=5, compute=himuon.FP32)
+    assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p256f), 0) > 0    # fp32: staged
+    p512 = himuon.params(512, (3.4445, -4.7750, 2.0315), steps=5)
+    need = lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p512), 0)
+    assert need > 512 * 512 * 4 * 64                        # at least the fp32 iterate of the 64 tiles
+    pc = himuon.params(512, (3.4445, -4.7750, 2.0315), steps=5, chunk_bytes=64 << 20)
     assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(pc), 0) <= 64 << 20
 
 
@@ -105,15 +109,17 @@ def test_per_matrix_tiles_on_the_host(lib):
     mats = (himuon.Mat * 3)(*[himuon.Mat(0x1000 * (i + 1), r, c, c, himuon.BF16) for i, (r, c) in enumerate(shapes)])
     one = lambda i: (himuon.Mat * 1)(mats[i])
     per = []
-    for i, T in enumerate((128, 256, 0)):
+    for i, T in enumerate((128, 512, 0)):
         per.append(lib.himuon_workspace_size(one(i), 1, None, ctypes.byref(himuon.params(T, Q, steps=5)),
                                              himuon.OP_NS_TILED if T > 0 else himuon.OP_NS_FULL))
     assert per[0] == 0 and per[1] > 0 and per[2] > 0
-    pt = himuon.params(128, Q, steps=5, tiles=[128, 256, 0])
+    pt = himuon.params(128, Q, steps=5, tiles=[128, 512, 0])
     for op in (himuon.OP_NS_TILED, himuon.OP_MOMENTUM_STEP):
         assert lib.himuon_workspace_size(mats, 3, None, ctypes.byref(pt), op) == max(per)
     # all on chip -> no workspace; ns_full ignores tiles
     assert lib.himuon_workspace_size(mats, 3, None, ctypes.byref(himuon.params(0, Q, steps=5, tiles=[128] * 3)),
+                                     himuon.OP_NS_TILED) == 0
+    assert lib.himuon_workspace_size(mats, 3, None, ctypes.byref(himuon.params(0, Q, steps=5, tiles=[128, 256, 64])),
                                      himuon.OP_NS_TILED) == 0
     full = lib.himuon_workspace_size(mats, 3, None, ctypes.byref(himuon.params(0, Q, steps=5)), himuon.OP_NS_FULL)
     assert lib.himuon_workspace_size(mats, 3, None, ctypes.byref(pt), himuon.OP_NS_FULL) == full

@@ -149,3 +149,22 @@ def test_wider_tiles_fit_the_budget_in_bf16(shape):
     """Tiles with both sides above 64 stay within both bounds with bf16 operands."""
     errb, svb = _worst_on_tiles(shape, to_bf16, range(24))
     assert errb <= BUDGET and svb <= 0.05, (errb, svb)
+
+
+def test_sixteen_step_list_needs_fp16_on_noisy_tiles():
+    """Five quintic then eleven cubic steps multiply a singular value near
+    zero by 3.4445^5 x 1.5^11 ~ 4e4: the noise floor of a low-rank-plus-noise
+    tile (normalised singular values down to ~1e-5) can end in the steep
+    middle of the map, where bf16 operand rounding moves it past the 0.05
+    bound and fp16 keeps it within."""
+    steps = [QUINTIC] * 5 + [CUBIC] * 11
+    c32 = [tuple(float(np.float32(v)) for v in s) for s in steps]
+    # the tile of the GPU test's 512 x 768 input whose smallest normalised
+    # singular value is 2e-5: the list maps it to 0.74, where the map is steep
+    X = to_bf16(inputs.low_rank_plus_noise(512, 768, inputs.sigma_inverse(32), 0.01, seed=19))[256:512, 512:768]
+    ref = oracle.ns_map(X, c32)
+    dev = {}
+    for name, rnd in (("bf16", to_bf16), ("fp16", to_fp16)):
+        got = scaled_operand_ns(X, steps, rnd)
+        dev[name] = np.abs(np.linalg.svd(got, compute_uv=False) - np.linalg.svd(ref, compute_uv=False)).max()
+    assert dev["bf16"] > 0.05 and dev["fp16"] <= 0.05, dev

@@ -12,8 +12,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhimuon.so")
-SOURCES = ["api.cu", "ns_resident.cu", "staged.cu", "static_scratch.cu"]
-HEADERS = ["ptx.cuh", "status.cuh", "layout.hpp", "resident.hpp", "staged.hpp"]
+SOURCES = ["api.cu", "ns_resident.cu", "ns_pair.cu", "staged.cu", "static_scratch.cu"]
+HEADERS = ["ptx.cuh", "status.cuh", "layout.hpp", "resident.hpp", "staged.hpp", "onchip.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I" + os.path.join(ROOT, "include"), "-I" + CSRC]

@@ -161,7 +161,7 @@ int check_call(const CallMats &cm, const himuon_split *splits) {
 }
 
 // ---------------------------------------------------------------- plans
-enum PathKind { kPathResident = 0, kPathStaged = 1 };
+enum PathKind { kPathResident = 0, kPathStaged = 1, kPathPair = 2 };
 
 struct TileClass {
   int64_t n, m;          // padded iterate shape (n <= m)
@@ -228,16 +228,33 @@ void *block_ptr(const himuon_mat &m, const HostBlock &b) {
 // when the call needs the staged path: fp32 arithmetic, non-bf16 storage,
 // misaligned rows, or tiles that are neither 128 x 128 (edge tiles smaller),
 // 64 x 64, 32 x 32, nor a whole block of at most 128 x 128.
-int resident_pack(const CallMats &cm, const std::vector<HostBlock> &blocks, const himuon_ns_params &p) {
-  if (p.compute == HIMUON_FP32) return 0;
+// The on-chip kernels read and write bf16 storage through 2-D tensor maps:
+// every role bf16, row pitch and block origins 16-byte aligned, 16-bit arithmetic.
+bool onchip_storage_ok(const CallMats &cm, const std::vector<HostBlock> &blocks, const himuon_ns_params &p) {
+  if (p.compute == HIMUON_FP32) return false;
   for (int r = 0; r < kNumRoles; ++r) {
     if (!cm.role[r]) continue;
     for (int32_t i = 0; i < cm.n; ++i) {
       const himuon_mat &m = cm.role[r][i];
-      if (m.dtype != HIMUON_BF16) return 0;
-      if ((m.ld * 2) % 16 != 0) return 0;
+      if (m.dtype != HIMUON_BF16) return false;
+      if ((m.ld * 2) % 16 != 0) return false;
     }
+    for (const HostBlock &b : blocks)
+      if (reinterpret_cast<uintptr_t>(block_ptr(cm.role[r][b.mat], b)) % 16 != 0) return false;
   }
+  return true;
+}
+
+// T = 256 runs on chip on CTA pairs (every block tiled at 256).
+bool pair_ok(const CallMats &cm, const std::vector<HostBlock> &blocks, const himuon_ns_params &p) {
+  if (p.tile != 256 || !onchip_storage_ok(cm, blocks, p)) return false;
+  for (const HostBlock &b : blocks)
+    if (b.T != 256) return false;
+  return true;
+}
+
+int resident_pack(const CallMats &cm, const std::vector<HostBlock> &blocks, const himuon_ns_params &p) {
+  if (!onchip_storage_ok(cm, blocks, p)) return 0;
   const int pack = (p.tile == 64 || p.tile == 32) ? 128 / p.tile : 1;
   for (const HostBlock &b : blocks) {
     if (pack > 1) {
@@ -245,10 +262,6 @@ int resident_pack(const CallMats &cm, const std::vector<HostBlock> &blocks, cons
     } else {
       const bool single = b.T >= std::max(b.rows, b.cols) && std::max(b.rows, b.cols) <= 128;
       if (!(b.T == 128 || single)) return 0;
-    }
-    for (int r = 0; r < kNumRoles; ++r) {
-      if (!cm.role[r]) continue;
-      if (reinterpret_cast<uintptr_t>(block_ptr(cm.role[r][b.mat], b)) % 16 != 0) return 0;
     }
   }
   return pack;
@@ -355,10 +368,12 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
   int rc = make_blocks(cm, splits, op == HIMUON_OP_NS_FULL ? 0 : p.tile, plan->blocks,
                        &plan->n_tiles);
   if (rc) return rc;
-  const int pack = (op != HIMUON_OP_GRAM_NS && !force_staged()) ? resident_pack(cm, plan->blocks, p) : 0;
-  const bool resident = pack > 0;
-  plan->path = resident ? kPathResident : kPathStaged;
-  plan->pack = resident ? pack : 1;
+  const bool onchip_ok = op != HIMUON_OP_GRAM_NS && !force_staged();
+  const bool pair = onchip_ok && pair_ok(cm, plan->blocks, p);
+  const int pack = (onchip_ok && !pair) ? resident_pack(cm, plan->blocks, p) : 0;
+  const bool resident = pack > 0 || pair;   // tiles on chip, read through tensor maps
+  plan->path = pair ? kPathPair : (pack > 0 ? kPathResident : kPathStaged);
+  plan->pack = pack > 0 ? pack : 1;
 
   std::vector<DevBlock> dblocks(plan->blocks.size());
   std::vector<CUtensorMap> tmaps;
@@ -371,7 +386,7 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
     d.tiles_c = static_cast<int32_t>(b.tiles_c);
     d.rows = static_cast<int32_t>(b.rows);
     d.cols = static_cast<int32_t>(b.cols);
-    d.T = resident ? 128 / pack : static_cast<int32_t>(b.T);
+    d.T = (resident && !pair) ? 128 / pack : static_cast<int32_t>(b.T);
     d.mat = b.mat;
     for (int r = 0; r < kNumRoles; ++r) {
       d.tmap[r] = -1;
@@ -382,7 +397,7 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
       d.dtype[r] = m.dtype;
       if (resident) {
         CUtensorMap tm;
-        if (!make_block_map(&tm, d.ptr[r], b.rows, b.cols, m.ld, pack)) return HIMUON_ERR_CUDA;
+        if (!make_block_map(&tm, d.ptr[r], b.rows, b.cols, m.ld, pair ? 1 : pack)) return HIMUON_ERR_CUDA;
         d.tmap[r] = static_cast<int32_t>(tmaps.size());
         tmaps.push_back(tm);
       }
@@ -412,8 +427,8 @@ int build_plan(int device, int op, const CallMats &cm, const himuon_split *split
   plan->d_tiles = reinterpret_cast<DevTile *>(static_cast<char *>(plan->dev) + sb + st);
   if (log_enabled()) {
     fprintf(stderr, "[himuon] plan: op=%d path=%s blocks=%zu tiles=%lld classes=%zu tmaps=%zu\n", op,
-            resident ? "resident" : "staged", plan->blocks.size(), (long long)plan->n_tiles, plan->classes.size(),
-            tmaps.size());
+            pair ? "pair" : (resident ? "resident" : "staged"), plan->blocks.size(), (long long)plan->n_tiles,
+            plan->classes.size(), tmaps.size());
     for (const TileClass &c : plan->classes)
       fprintf(stderr, "[himuon]   class n=%lld m=%lld tiles=%zu padded=%d thin=%d compute=%d\n", (long long)c.n,
               (long long)c.m, c.tiles.size(), (int)c.padded, (int)c.thin, class_compute(c, op, p.compute));
@@ -781,6 +796,10 @@ int run_resident(const Plan &plan, int op, const himuon_ns_params &p, float mu, 
   make_resident_steps(a, p.coeffs, p.steps);
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, plan.device);
+  if (plan.path == kPathPair) {   // one 256 x 256 tile per CTA pair at a time
+    const int pairs = static_cast<int>(std::min<int64_t>(sms / 2, plan.n_tiles));
+    return launch_ns_pair(a, pairs, stream) == cudaSuccess ? HIMUON_OK : HIMUON_ERR_CUDA;
+  }
   const int64_t n_super = (plan.n_tiles + plan.pack - 1) / plan.pack;
   const int64_t want = (n_super + 1) / 2;
   const int grid = static_cast<int>(std::min<int64_t>(sms, want));
@@ -810,7 +829,7 @@ int prepare(int op, const CallMats &cm, const himuon_split *splits, const himuon
   pr.p = *p;
   pr.has_w = op == HIMUON_OP_MOMENTUM_STEP && cm.role[kRoleW];
   pr.has_o = cm.role[kRoleOut] != nullptr;
-  if (pr.plan->path == kPathResident) return HIMUON_OK;
+  if (pr.plan->path != kPathStaged) return HIMUON_OK;
   const int64_t need = staged_ws_bytes(*pr.plan, op, p->compute);
   if (!ws || static_cast<int64_t>(ws_bytes) < need) return HIMUON_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return HIMUON_ERR_ALIGNMENT;
@@ -819,7 +838,7 @@ int prepare(int op, const CallMats &cm, const himuon_split *splits, const himuon
 
 int launch(const Prepared &pr, float mu, float lr, void *ws, size_t ws_bytes, void *stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (pr.plan->path == kPathResident) return run_resident(*pr.plan, pr.op, pr.p, mu, lr, pr.has_w, pr.has_o, s);
+  if (pr.plan->path != kPathStaged) return run_resident(*pr.plan, pr.op, pr.p, mu, lr, pr.has_w, pr.has_o, s);
   return run_staged(*pr.plan, pr.op, pr.p, mu, lr, ws, ws_bytes, s);
 }
 
@@ -906,7 +925,8 @@ int64_t workspace_one(const CallMats &cm, const himuon_split *splits, const himu
   const int64_t tile = op == HIMUON_OP_NS_FULL ? 0 : p.tile;
   int rc = make_blocks(cm, splits, tile, blocks, &n_tiles);
   if (rc) return rc;
-  if (op != HIMUON_OP_GRAM_NS && !force_staged() && resident_pack(cm, blocks, p) > 0) return 0;
+  if (op != HIMUON_OP_GRAM_NS && !force_staged() && (pair_ok(cm, blocks, p) || resident_pack(cm, blocks, p) > 0))
+    return 0;
   // staged: one tile of the largest class is the minimum; a full chunk of every
   // class makes the call run in one chunk per class.
   int64_t need = 0;

@@ -1,0 +1,538 @@
+// ns_pair.cu -- tiled NS with 256 x 256 tiles kept on chip for all K steps,
+// one tile per CTA pair.
+//
+// The map ("Gram Newton-Schulz" page, sec. 3, Algorithm 1, applied per tile as
+// in the "Hierarchical Muon" abstract) on tiles of T = 256: normalise by
+// (||X||_F + eps), then per step A = X X^T, B = b A + c A^2, X = a X + B X.
+// Ragged edge tiles are zero-padded to 256 x 256 (the same map, as on the
+// 128-tile kernel: a zero border stays zero and NS(X^T) = NS(X)^T).
+//
+// A 256 x 256 tile does not fit one SM's tensor memory twice (two fp32 256 x 256
+// accumulators are 2 x 256 KB), so each tile runs on a pair of CTAs in a
+// cluster of two: CTA c owns rows 128c .. 128c + 127 of the tile and of every
+// 256 x 256 product, in its own TMEM (256 columns for D_P, 256 for D_X).  The
+// even CTA issues every MMA as a pair MMA (cta_group::2, M = 256, N = 256):
+// each CTA supplies its 128 rows of the A operand from its TMEM and 128 of the
+// N rows of the B operand from its shared memory.  With the iterate carried
+// scaled by g = sqrt|c/b| as on the 128-tile kernel:
+//   MMA1  D_P  = Xg Xg^T           A: Xg (own rows, packed in D_X)   B: own rows of Xg (K-major)
+//   MMA2  D_P += sign(c/b) S S^T    A: S  (own rows, packed in D_X)   B: own rows of S  (K-major)
+//   MMA3  D_X  = Bop Xg             A: Bop (own rows, packed in D_P)  B: columns 128c .. 128c+127 of Xg,
+//                                                                        all 256 rows (MN-major)
+// so only MMA3's B operand needs the partner's rows: after each conversion of
+// the iterate every CTA writes its rows' values of the partner's column half
+// into the partner's shared memory (32 KB per step, distributed shared memory),
+// and each tile's norm is the sum of the two CTAs' partial sums.  Operands are
+// ready for a job when all 16 warps of both CTAs have arrived on the even
+// CTA's ready barrier; the even CTA's issuing thread then issues the job's 16
+// MMAs and commits them to the MMA barrier of both CTAs (multicast commit).
+// Shared memory per CTA: X_s (128 rows x 256, K-major, 64 KB), S_s (same;
+// also G / M' in the prologue and W / W' in the epilogue), X_mn (256 rows x
+// this CTA's 128 columns, MN-major, 64 KB).
+//
+// Operand type per tile as on the 128-tile kernel: a bf16 call rounds the
+// operands of a tile with a short side of at most 64 to fp16 (unless its
+// normalised norm is below 2^-10).  Every wait is bounded; a CTA that gives up
+// raises its own and its partner's abort flag, and the pair meets at the end
+// in one cluster barrier, after which each CTA releases its TMEM.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "layout.hpp"
+#include "onchip.cuh"
+#include "ptx.cuh"
+#include "resident.hpp"
+
+namespace himuon {
+
+namespace {
+
+using namespace onchip;
+
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr uint32_t kChunk = 16384;      // 128 rows x 64 columns of 16-bit values, 128-byte swizzle
+constexpr uint32_t kOffX = 0;           // X_s: own rows, K-major, 4 chunks
+constexpr uint32_t kOffS = 65536;       // S_s: own rows, K-major, 4 chunks
+constexpr uint32_t kOffMN = 131072;     // X_mn: all 256 rows of this CTA's 128 columns, MN-major
+constexpr uint32_t kMnHalf = 32768;     // its two 64-column halves (256 rows x 128 bytes each)
+constexpr uint32_t kOffBars = 196608;
+constexpr uint32_t kSmemBytes = kOffBars + 512 + 1024;   // + alignment slack
+
+struct PairSmem {
+  uint8_t *base;
+  __device__ uint8_t *x() const { return base + kOffX; }
+  __device__ uint8_t *s() const { return base + kOffS; }
+  __device__ uint8_t *mn() const { return base + kOffMN; }
+  __device__ uint64_t *bar(int i) const { return reinterpret_cast<uint64_t *>(base + kOffBars) + i; }
+  __device__ uint64_t *bar_ld() const { return bar(0); }     // M (or input) and G landed
+  __device__ uint64_t *bar_w() const { return bar(1); }      // W landed
+  __device__ uint64_t *bar_mma() const { return bar(2); }    // the pair's MMA job finished (multicast commit)
+  __device__ uint64_t *bar_ready() const { return bar(3); }  // even CTA: both CTAs' operands of the next job written
+  __device__ uint64_t *bar_pro() const { return bar(4); }    // prologue: M' and partial norms of this CTA written
+  __device__ uint64_t *bar_norm() const { return bar(5); }   // the partner's partial norm landed
+  __device__ uint64_t *bar_epi() const { return bar(6); }    // epilogue: W' / O staged
+  __device__ uint64_t *bar_never() const { return bar(7); }  // never arrived on (stall self-test)
+  __device__ float *red() const { return reinterpret_cast<float *>(base + kOffBars + 64); }   // kWarps floats
+  __device__ float *peer_norm() const { return reinterpret_cast<float *>(base + kOffBars + 128); }
+  __device__ uint32_t *tmem_slot() const { return reinterpret_cast<uint32_t *>(base + kOffBars + 132); }
+  __device__ volatile int *abort_flag() const { return reinterpret_cast<volatile int *>(base + kOffBars + 136); }
+  __device__ TileCoord *coord(int i) const { return reinterpret_cast<TileCoord *>(base + kOffBars + 192) + i; }
+};
+
+// Bounded wait (cluster-scope acquire: some phases complete by the partner's
+// arrivals).  On a timeout it records HIMUON_ERR_TIMEOUT and raises the abort
+// flag of both CTAs of the pair; it gives up as soon as the flag is raised.
+__device__ __forceinline__ bool pair_wait(uint64_t *bar, uint32_t parity, const PairSmem &sm, uint32_t peer,
+                                          int *status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 255u) == 0) {
+      if (*sm.abort_flag()) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+  }
+  set_status(status, HIMUON_ERR_TIMEOUT);
+  *sm.abort_flag() = 1;
+  st_cluster_u32(mapa_shared(smem_u32(const_cast<int *>(sm.abort_flag())), peer), 1u);
+  return false;
+}
+
+// Byte offset of 16-byte chunk `c8` (0..31) of row `r` in a K-major operand of
+// 256 columns: four 64-column, 128-byte-swizzled chunks.
+__device__ __forceinline__ uint32_t kmaj_off(uint32_t r, uint32_t c8) {
+  return (c8 >> 3) * kChunk + sw128_off(r, c8 & 7u);
+}
+// Byte offset of 16-byte chunk `c8` (0..15) of K-row `k` (0..255) in X_mn.
+__device__ __forceinline__ uint32_t mn_off(uint32_t k, uint32_t c8) {
+  return (c8 >> 3) * kMnHalf + sw128_off(k, c8 & 7u);
+}
+
+// This thread's 64 columns (chunk cb) of row r of a 256-column fp32 TMEM
+// region -> r(scale * v): packed in place to TMEM columns [64 cb, 64 cb + 32)
+// of `pk` (the A operand), and to the K-major shared operand `kdst` (nullptr:
+// none).  With `mn` the values also go to X_mn of the CTA that owns these
+// columns (cb / 2; the partner's through distributed shared memory), as row
+// 128 c + r.
+template <int F>
+__device__ __forceinline__ void pair_row_to_op(uint32_t src, uint32_t pk, uint8_t *kdst, uint32_t r, uint32_t cb,
+                                               float scale, bool mn, uint32_t mn_addr, uint32_t krow) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float v[32];
+    tmem_ld32(src + 64u * cb + 32u * i, v);
+    tmem_wait_ld();
+    uint32_t p[16];
+    if (scale != 1.f) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) p[e] = pack2_op<F>(v[2 * e] * scale, v[2 * e + 1] * scale);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) p[e] = pack2_op<F>(v[2 * e], v[2 * e + 1]);
+    }
+    tmem_st16(pk + 64u * cb + 16u * i, p);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 u = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+      const uint32_t c8 = 8u * cb + 4u * i + j;            // 16-byte chunk of the 256-column row
+      if (kdst) *reinterpret_cast<uint4 *>(kdst + kmaj_off(r, c8)) = u;
+      if (mn) st_cluster_v4(mn_addr + mn_off(krow, c8 & 15u), u);
+    }
+  }
+  tmem_wait_st();
+}
+
+// Bop = r(beta * D_P + diag * I) for this thread's 64 columns, packed in place.
+// Row r of CTA c is row 128 c + r of the tile: its diagonal element sits in
+// chunk (128 c + r) / 64 at position (128 c + r) % 64.
+template <int F>
+__device__ __forceinline__ void pair_row_to_bop(uint32_t taddr, uint32_t grow, uint32_t cb, float beta, float diag) {
+  const bool dchunk = (grow >> 6) == cb;
+  const uint32_t dpos = grow & 63u;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float v[32];
+    tmem_ld32(taddr + 64u * cb + 32u * i, v);
+    tmem_wait_ld();
+    uint32_t p[16];
+    if (dchunk && (dpos >> 5) == static_cast<uint32_t>(i)) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float a0 = fmaf(beta, v[2 * e], (dpos & 31u) == 2u * e ? diag : 0.f);
+        const float a1 = fmaf(beta, v[2 * e + 1], (dpos & 31u) == 2u * e + 1u ? diag : 0.f);
+        p[e] = pack2_op<F>(a0, a1);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) p[e] = pack2_op<F>(beta * v[2 * e], beta * v[2 * e + 1]);
+    }
+    tmem_st16(taddr + 64u * cb + 16u * i, p);
+  }
+  tmem_wait_st();
+}
+
+enum Job { kJobGram = 0, kJobSquare = 1, kJobUpdate = 2 };
+
+// TMEM column of the packed A operand for k-step kk (K elements 16 kk .. +15)
+__device__ __forceinline__ uint32_t acol(int kk) { return 64u * (kk >> 2) + 8u * (kk & 3); }
+
+// The even CTA's issuing thread: the job's sixteen 256x256x16 pair MMAs,
+// committed to the MMA barrier of both CTAs.
+template <int JOB>
+__device__ __forceinline__ void pair_issue(const PairSmem &sm, uint32_t tmem, const ResidentStep *st, bool f16) {
+  tc_fence_after();
+  const uint32_t dP = tmem, dX = tmem + 256u;
+  const uint64_t tk = sw128_desc(0, 16, 1024);
+  if (JOB == kJobGram) {
+    const uint32_t x4 = smem_u32(sm.x()) >> 4;
+    const uint32_t id = f16 ? idesc_f16(256, 256, 0, 0, 0, 0) : idesc_f16(256, 256, 1, 0, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk)
+      mma_ts_pair(dP, dX + acol(kk), tk + x4 + (((kk >> 2) * kChunk + (kk & 3) * 32) >> 4), id, kk > 0);
+  } else if (JOB == kJobSquare) {
+    const uint32_t s4 = smem_u32(sm.s()) >> 4;
+    const uint32_t id = idesc_f16(256, 256, f16 ? 0 : 1, 0, 0, st->neg2);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk)
+      mma_ts_pair(dP, dX + acol(kk), tk + s4 + (((kk >> 2) * kChunk + (kk & 3) * 32) >> 4), id, st->acc2 | (kk > 0));
+  } else {
+    const uint32_t m4 = smem_u32(sm.mn()) >> 4;
+    const uint64_t tmn = sw128_desc(0, kMnHalf, 1024);
+    const uint32_t id = f16 ? idesc_f16(256, 256, 0, 0, 1, 0) : idesc_f16(256, 256, 1, 0, 1, 0);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) mma_ts_pair(dX, dP + acol(kk), tmn + m4 + ((kk * 2048) >> 4), id, kk > 0);
+  }
+  mma_commit_pair(sm.bar_mma(), 3);
+}
+
+// Boxes of this CTA's 128 rows of a tile: 64 columns x 128 rows each, at
+// (x0 + 64 j, y0 + 128 c); boxes wholly past the block's last column or row
+// are skipped on stores (loads read zeros there).
+__device__ __forceinline__ void load_rows(const CUtensorMap *m, uint8_t *dst, const TileCoord &t, uint32_t c,
+                                          uint64_t *bar) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) tma_load_2d(dst + j * kChunk, m, t.x0 + 64 * j, t.y0 + 128 * static_cast<int>(c), bar);
+}
+__device__ __forceinline__ void store_rows(const CUtensorMap *m, const uint8_t *src, const TileCoord &t, uint32_t c) {
+  if (128 * static_cast<int>(c) >= t.h) return;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (64 * j < t.w) tma_store_2d(m, src + j * kChunk, t.x0 + 64 * j, t.y0 + 128 * static_cast<int>(c));
+}
+__device__ __forceinline__ void prefetch_rows(const CUtensorMap *m, const TileCoord &t, uint32_t c) {
+  if (128 * static_cast<int>(c) >= t.h) return;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (64 * j < t.w) tma_prefetch_l2_2d(m, t.x0 + 64 * j, t.y0 + 128 * static_cast<int>(c));
+}
+
+__device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tmem) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t c = cluster_ctarank();           // 0: even CTA (issues the MMAs), 1: odd CTA
+  const uint32_t peer = c ^ 1u;
+  const uint32_t q = static_cast<uint32_t>(warp & 3);   // TMEM lane quarter
+  const uint32_t cb = static_cast<uint32_t>(warp >> 2); // 64-column chunk of the 256-column row
+  const uint32_t r = q * 32 + lane;               // row among this CTA's 128
+  const uint32_t grow = 128u * c + r;             // row of the tile
+  const uint32_t tP = tmem + ((q * 32) << 16);    // this warp's lanes of D_P (columns 0..255)
+  const uint32_t tX = tP + 256u;                  // ... and of D_X (columns 256..511)
+  uint8_t *Xs = sm.x(), *Ss = sm.s();
+  const bool step_mode = a.mode == 1;
+  const bool has_w = step_mode && a.has_w;
+  const bool leader = c == 0 && threadIdx.x == 0;
+  const bool tma = threadIdx.x == 0;              // this CTA's TMA-issuing thread
+  // X_mn of the CTA that owns this thread's columns (itself or the partner)
+  const uint32_t mn_owner = cb >> 1;
+  const uint32_t mn_addr = mapa_shared(smem_u32(sm.mn()), mn_owner);
+  // the even CTA's ready barrier (local for c = 0)
+  const uint32_t ready_addr = mapa_shared(smem_u32(sm.bar_ready()), 0);
+  const uint32_t peer_norm_addr = mapa_shared(smem_u32(sm.peer_norm()), peer);
+  const uint32_t peer_norm_bar = mapa_shared(smem_u32(sm.bar_norm()), peer);
+  const int64_t n_pairs = gridDim.x / 2;
+  const int64_t pair = blockIdx.x / 2;
+  uint32_t it = 0, job = 0;
+  uint32_t ld_armed = 0, ld_seen = 0, w_armed = 0, w_seen = 0, mma_issued = 0;
+  TileCoord *cur = sm.coord(0), *nxt = sm.coord(1);
+  if (a.test_stall && pair == 0) pair_wait(sm.bar_never(), 0, sm, peer, a.status);
+  if (tma) *cur = decode_tile(a, nullptr, pair);
+  __syncthreads();
+  bool bad = *sm.abort_flag() != 0;
+
+  for (int64_t tile = pair; tile < a.n_tiles && !bad; tile += n_pairs, ++it) {
+    if (tma) {
+      bulk_wait_read0();   // the previous tile's stores have finished reading X_s / S_s
+      mbar_arrive_expect_tx(sm.bar_ld(), (step_mode ? 2u : 1u) * 4u * kChunk);
+      load_rows(a.tmaps + cur->tm[kRoleIn], Xs, *cur, c, sm.bar_ld());
+      if (step_mode) load_rows(a.tmaps + cur->tm[kRoleG], Ss, *cur, c, sm.bar_ld());
+      ++ld_armed;
+    }
+    __syncwarp();
+    bad = !pair_wait(sm.bar_ld(), it & 1u, sm, peer, a.status);
+    if (tma && !bad) ++ld_seen;
+    if (__any_sync(0xffffffffu, bad)) break;
+
+    // ---- prologue: M' = mu M + G (or the plain input), this CTA's ||.||_F^2, fp32 copy to D_X
+    float sumsq = 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float v[32];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t c8 = 8 * cb + 4 * i + k;
+        float m[8];
+        unpack8(*reinterpret_cast<const uint4 *>(Xs + kmaj_off(r, c8)), m);
+        if (step_mode) {
+          float g[8];
+          unpack8(*reinterpret_cast<const uint4 *>(Ss + kmaj_off(r, c8)), g);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m[e] = fmaf(a.mu, m[e], g[e]);
+          *reinterpret_cast<uint4 *>(Ss + kmaj_off(r, c8)) = pack8_bf16(m);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[8 * k + e] = m[e];
+          sumsq = fmaf(m[e], m[e], sumsq);
+        }
+      }
+      tmem_st32(tX + 64 * cb + 32 * i, v);
+    }
+    tmem_wait_st();
+    sumsq = warp_sum(sumsq);
+    if (lane == 0) sm.red()[warp] = sumsq;
+    if (step_mode) fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.bar_pro());
+    bad = !pair_wait(sm.bar_pro(), it & 1u, sm, peer, a.status);
+    if (__any_sync(0xffffffffu, bad)) break;
+    tc_fence_after();
+    float own = 0.f;   // this CTA's ||rows||^2, summed in one order by every thread
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) own += sm.red()[w];
+    if (tma) {
+      if (step_mode) {
+        store_rows(a.tmaps + cur->tm[kRoleIn], Ss, *cur, c);
+        bulk_commit();
+      }
+      st_cluster_f32(peer_norm_addr, own);   // the partner's half of the tile norm
+      mbar_arrive_cluster(peer_norm_bar);
+    }
+    __syncwarp();
+    bad = !pair_wait(sm.bar_norm(), it & 1u, sm, peer, a.status);
+    if (__any_sync(0xffffffffu, bad)) break;
+    const float total = own + *sm.peer_norm();      // the same value in both CTAs (a + b = b + a)
+    const float nrm = sqrtf(total);
+    const float rho = (nrm + a.eps) * a.safety;
+    bool f16 = a.op_fmt == 0;
+    if (!f16 && a.f16_small)
+      f16 = min(cur->h, cur->w) <= 64 && !(total > 0.f && nrm < kTinyNorm * rho);
+
+    // ---- operand g_0 X_0 = r(g_0 M' / rho): X_s, packed in D_X, and X_mn of the column owner
+    if (f16) pair_row_to_op<0>(tX, tX, Xs, r, cb, a.gamma0 / rho, true, mn_addr, grow);
+    else pair_row_to_op<1>(tX, tX, Xs, r, cb, a.gamma0 / rho, true, mn_addr, grow);
+    // M' must have left S_s before the first conversion (after MMA1) overwrites
+    // it: MMA1 waits for this thread's arrival below
+    if (step_mode && tma) bulk_wait_read0();
+    fence_proxy_async_cluster();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(ready_addr);
+    if (leader) {
+      bad = !pair_wait(sm.bar_ready(), job & 1u, sm, peer, a.status);
+      if (!bad) {
+        pair_issue<kJobGram>(sm, tmem, nullptr, f16);
+        ++mma_issued;
+      }
+    }
+    if (tma) {   // next tile of this pair, while MMA1 runs
+      *nxt = decode_tile(a, nullptr, tile + n_pairs);
+      if (nxt->blk >= 0) {
+        prefetch_rows(a.tmaps + nxt->tm[kRoleIn], *nxt, c);
+        if (step_mode) prefetch_rows(a.tmaps + nxt->tm[kRoleG], *nxt, c);
+        if (has_w) prefetch_rows(a.tmaps + nxt->tm[kRoleW], *nxt, c);
+      }
+    }
+    if (__any_sync(0xffffffffu, bad)) break;
+
+    bool stop = false;
+    for (int t = 0; t < a.K && !stop; ++t) {
+      const ResidentStep *stp = &a.step[t];
+      // after MMA1: S = r(s D_P) to S_s and (packed) to D_X
+      bad = !pair_wait(sm.bar_mma(), job++ & 1u, sm, peer, a.status);
+      if ((stop = __any_sync(0xffffffffu, bad))) break;
+      tc_fence_after();
+      if (f16) pair_row_to_op<0>(tP, tX, Ss, r, cb, stp->s, false, 0, 0);
+      else pair_row_to_op<1>(tP, tX, Ss, r, cb, stp->s, false, 0, 0);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(ready_addr);
+      if (leader) {
+        bad = !pair_wait(sm.bar_ready(), job & 1u, sm, peer, a.status);
+        if (!bad) {
+          pair_issue<kJobSquare>(sm, tmem, stp, f16);
+          ++mma_issued;
+        }
+      }
+      if ((stop = __any_sync(0xffffffffu, bad))) break;
+      // after MMA2: Bop = r(beta D_P + a I), packed in D_P
+      bad = !pair_wait(sm.bar_mma(), job++ & 1u, sm, peer, a.status);
+      if ((stop = __any_sync(0xffffffffu, bad))) break;
+      tc_fence_after();
+      if (t + 1 == a.K && has_w && tma) {   // S_s is free for good: W lands there for the epilogue
+        mbar_arrive_expect_tx(sm.bar_w(), 4u * kChunk);
+        load_rows(a.tmaps + cur->tm[kRoleW], Ss, *cur, c, sm.bar_w());
+        ++w_armed;
+      }
+      if (f16) pair_row_to_bop<0>(tP, grow, cb, stp->beta, stp->a);
+      else pair_row_to_bop<1>(tP, grow, cb, stp->beta, stp->a);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(ready_addr);
+      if (leader) {
+        bad = !pair_wait(sm.bar_ready(), job & 1u, sm, peer, a.status);
+        if (!bad) {
+          pair_issue<kJobUpdate>(sm, tmem, stp, f16);
+          ++mma_issued;
+        }
+      }
+      if ((stop = __any_sync(0xffffffffu, bad))) break;
+      // after MMA3: next operand r(xr D_X) = g_{t+1} X_{t+1}: X_s, packed in D_X, X_mn
+      bad = !pair_wait(sm.bar_mma(), job++ & 1u, sm, peer, a.status);
+      if ((stop = __any_sync(0xffffffffu, bad))) break;
+      tc_fence_after();
+      if (t + 1 < a.K) {
+        if (f16) pair_row_to_op<0>(tX, tX, Xs, r, cb, stp->xr, true, mn_addr, grow);
+        else pair_row_to_op<1>(tX, tX, Xs, r, cb, stp->xr, true, mn_addr, grow);
+        fence_proxy_async_cluster();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ready_addr);
+        if (leader) {
+          bad = !pair_wait(sm.bar_ready(), job & 1u, sm, peer, a.status);
+          if (!bad) {
+            pair_issue<kJobGram>(sm, tmem, nullptr, f16);
+            ++mma_issued;
+          }
+        }
+        if ((stop = __any_sync(0xffffffffu, bad))) break;
+      }
+    }
+    if (stop) break;
+
+    // ---- epilogue: O = D_X / g;  W <- W - lr O   (this CTA's rows)
+    if (has_w) {
+      bad = !pair_wait(sm.bar_w(), it & 1u, sm, peer, a.status);
+      if (tma && !bad) ++w_seen;
+      if (__any_sync(0xffffffffu, bad)) break;
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float v[32];
+      tmem_ld32(tX + 64 * cb + 32 * i, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t off = kmaj_off(r, 8 * cb + 4 * i + k);
+        const float *o = v + 8 * k;   // gamma_{K-1} O
+        if (a.has_o) {
+          float ov[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ov[e] = a.oscale * o[e];
+          *reinterpret_cast<uint4 *>(Xs + off) = pack8_bf16(ov);
+        }
+        if (has_w) {
+          const float lro = -a.lr * a.oscale;
+          float w[8];
+          unpack8(*reinterpret_cast<const uint4 *>(Ss + off), w);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = fmaf(lro, o[e], w[e]);
+          *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(w);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.bar_epi());
+    if (tma) {
+      bad = !pair_wait(sm.bar_epi(), it & 1u, sm, peer, a.status);
+      if (!bad) {
+        if (a.has_o) store_rows(a.tmaps + cur->tm[kRoleOut], Xs, *cur, c);
+        if (has_w) store_rows(a.tmaps + cur->tm[kRoleW], Ss, *cur, c);
+        bulk_commit();
+      }
+      *cur = *nxt;
+    }
+    // The next tile's loads (issued by the TMA thread after its stores have
+    // read X_s / S_s) gate everyone's next prologue.
+    if (__any_sync(0xffffffffu, bad)) break;
+  }
+  if (tma) {
+    // After an abort: wait (bounded) for this CTA's loads still in flight.
+    for (; ld_seen < ld_armed; ++ld_seen) mbar_wait(sm.bar_ld(), ld_seen & 1u, a.status);
+    for (; w_seen < w_armed; ++w_seen) mbar_wait(sm.bar_w(), w_seen & 1u, a.status);
+    bulk_wait0();
+  }
+  if (leader && mma_issued > 0) {
+    // every pair MMA issued has finished before the pair releases its memory
+    mbar_wait(sm.bar_mma(), (mma_issued - 1u) & 1u, a.status);
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    ns_pair_kernel(const __grid_constant__ ResidentArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  PairSmem sm;
+  sm.base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(sm.bar_ld(), 1);
+    mbar_init(sm.bar_w(), 1);
+    mbar_init(sm.bar_mma(), 1);
+    mbar_init(sm.bar_ready(), 2 * kWarps);
+    mbar_init(sm.bar_pro(), kWarps);
+    mbar_init(sm.bar_norm(), 1);
+    mbar_init(sm.bar_epi(), kWarps);
+    mbar_init(sm.bar_never(), 1);
+    *sm.abort_flag() = 0;
+    *sm.peer_norm() = 0.f;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(sm.tmem_slot(), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();   // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem = *sm.tmem_slot();
+
+  pair_main(args, sm, tmem);
+
+  tc_fence_before();
+  cluster_sync_all();   // neither CTA releases its memory while the partner may still use it
+  tc_fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+}  // namespace
+
+int pair_smem_bytes() { return static_cast<int>(kSmemBytes); }
+
+cudaError_t launch_ns_pair(const ResidentArgs &args, int pairs, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(ns_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  count_launch();
+  ns_pair_kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(args);
+  return cudaGetLastError();
+}
+
+}  // namespace himuon

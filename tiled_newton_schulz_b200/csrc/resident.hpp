@@ -46,6 +46,9 @@ struct ResidentArgs {
 void make_resident_steps(ResidentArgs &args, const float *coeffs, int K);
 
 int resident_smem_bytes();
+// 256 x 256 tiles on CTA pairs (clusters of two): `pairs` tiles in flight.
+int pair_smem_bytes();
+cudaError_t launch_ns_pair(const ResidentArgs &args, int pairs, cudaStream_t stream);
 int resident_max_smem_blocks();
 cudaError_t launch_ns_resident(const ResidentArgs &args, int grid, cudaStream_t stream);
 
