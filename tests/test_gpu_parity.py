@@ -415,3 +415,73 @@ def test_pair_momentum_step(hm):
         got = to_np(o[i])
         wexp = w0[i] - lr32 * got
         assert np.all(np.abs(to_np(w[i]) - wexp) <= bf16_ulp(wexp) + lr32 * bf16_ulp(got) + 1e-12)
+
+
+# ---- many tiles per CTA (pair): the loop over tiles, with the next tile's
+# loads in flight during the current tile's last step
+LOOP_SHAPES = [(520, 600), (40, 700), (300, 130)]   # ragged, thin (fp16 operands in bf16 calls), tall
+_LOOP_REF = {}
+
+
+def _loop_inputs():
+    rng = np.random.default_rng(31)
+    w = [0.02 * rng.standard_normal(sh) for sh in LOOP_SHAPES]
+    m = [inputs.low_rank_plus_noise(*sh, inputs.sigma_inverse(16), 0.01, seed=700 + i) for i, sh in enumerate(LOOP_SHAPES)]
+    g = [inputs.low_rank_plus_noise(*sh, inputs.sigma_inverse(16), 0.01, seed=800 + i) for i, sh in enumerate(LOOP_SHAPES)]
+    bf = lambda a: to_np(torch.from_numpy(a).to(torch.bfloat16))
+    return [bf(x) for x in w], [bf(x) for x in m], [bf(x) for x in g]
+
+
+def _loop_reference(T, mode):
+    key = (T, mode)
+    if key not in _LOOP_REF:
+        w0, m0, g0 = _loop_inputs()
+        if mode == "ns":
+            _LOOP_REF[key] = [oracle.ns_tiled(x, T, C32) for x in m0]
+        else:
+            _LOOP_REF[key] = [oracle.momentum_step(w0[i], m0[i], g0[i], 0.95, 0.02, T, C32)
+                              for i in range(len(LOOP_SHAPES))]
+    return _LOOP_REF[key]
+
+
+@pytest.mark.parametrize("mode", ["ns", "step", "step_out"])
+@pytest.mark.parametrize("T,ctas", [(256, 2), (256, 6), (128, 1), (128, 3)])
+def test_onchip_tile_loop(hm, monkeypatch, T, ctas, mode):
+    """HIMUON_MAX_CTAS caps the launch so that every CTA (pair) runs many
+    tiles of three matrices in its loop: tile coordinates, loads issued
+    during the previous tile's last step, per-tile operand type (the thin
+    matrix's tiles take fp16 operands), ragged edges and the fused step's
+    three outputs must all follow the tile being processed."""
+    monkeypatch.setenv("HIMUON_MAX_CTAS", str(ctas))
+    w0, m0, g0 = _loop_inputs()
+    ref = _loop_reference(T, "ns" if mode == "ns" else "step")
+    p = hm.params(T, QUINTIC, steps=5)
+    if mode == "ns":
+        x = [dev(a, torch.bfloat16) for a in m0]
+        y = [torch.empty_like(a) for a in x]
+        hm.ns_tiled(x, y, p)
+        assert hm.device_status() == 0
+        for i in range(len(LOOP_SHAPES)):
+            check16(to_np(y[i]), ref[i], T)
+        return
+    w = [dev(a, torch.bfloat16) for a in w0]
+    m = [dev(a, torch.bfloat16) for a in m0]
+    g = [dev(a, torch.bfloat16) for a in g0]
+    o = [torch.empty_like(a) for a in m] if mode == "step_out" else None
+    hm.momentum_step(w, m, g, 0.95, 0.02, p, update_out=o)
+    assert hm.device_status() == 0
+    lr32 = float(np.float32(0.02))
+    for i in range(len(LOOP_SHAPES)):
+        W2, M2, O = ref[i]
+        assert np.all(np.abs(to_np(m[i]) - M2) <= bf16_ulp(M2)), i
+        wg = to_np(w[i])
+        if o is not None:
+            got = to_np(o[i])
+            check16(got, O, T)
+            wexp = w0[i] - lr32 * got
+            assert np.all(np.abs(wg - wexp) <= bf16_ulp(wexp) + lr32 * bf16_ulp(got) + 1e-12)
+        else:
+            for (r, c, h, ww) in tiles(*LOOP_SHAPES[i], T):
+                sl = np.s_[r:r + h, c:c + ww]
+                bound = np.linalg.norm(0.5 * bf16_ulp(W2[sl])) + lr32 * TOL16 * np.linalg.norm(O[sl])
+                assert np.linalg.norm(wg[sl] - W2[sl]) <= bound, (i, r, c)

@@ -64,6 +64,15 @@ bool force_staged() {
   return e && strcmp(e, "staged") == 0;
 }
 
+// HIMUON_MAX_CTAS=n caps the CTAs of an on-chip launch (tests only: with a
+// few CTAs every CTA, or CTA pair, runs many tiles in its loop, the way the
+// large calls do); read on every call, 0 or unset = one per SM.
+int max_ctas() {
+  const char *e = getenv("HIMUON_MAX_CTAS");
+  const int v = e ? atoi(e) : 0;
+  return v > 0 ? v : 0;
+}
+
 size_t elem_size(int32_t dt) { return dt == HIMUON_FP32 ? 4 : 2; }
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
@@ -796,6 +805,7 @@ int run_resident(const Plan &plan, int op, const himuon_ns_params &p, float mu, 
   make_resident_steps(a, p.coeffs, p.steps);
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, plan.device);
+  if (const int cap = max_ctas()) sms = std::max(2, std::min(sms, cap));
   if (plan.path == kPathPair) {   // one 256 x 256 tile per CTA pair at a time
     const int pairs = static_cast<int>(std::min<int64_t>(sms / 2, plan.n_tiles));
     return launch_ns_pair(a, pairs, stream) == cudaSuccess ? HIMUON_OK : HIMUON_ERR_CUDA;

@@ -114,12 +114,14 @@ __device__ __forceinline__ uint32_t mn_off(uint32_t k, uint32_t c8) {
 // This thread's 64 columns (chunk cb) of row r of a 256-column fp32 TMEM
 // region -> r(scale * v): packed in place to TMEM columns [64 cb, 64 cb + 32)
 // of `pk` (the A operand), and to the K-major shared operand `kdst` (nullptr:
-// none).  With `mn` the values also go to X_mn of the CTA that owns these
-// columns (cb / 2; the partner's through distributed shared memory), as row
-// 128 c + r.
-template <int F>
+// none).  MN says where the values also go as row `krow` (= 128 c + r) of X_mn
+// of the CTA that owns these columns (cb / 2): kMnNone, kMnLocal (this CTA:
+// `mn_local`), kMnRemote (the partner, through distributed shared memory at
+// `mn_remote`).
+enum MnTarget { kMnNone = 0, kMnLocal = 1, kMnRemote = 2 };
+template <int F, int MN>
 __device__ __forceinline__ void pair_row_to_op(uint32_t src, uint32_t pk, uint8_t *kdst, uint32_t r, uint32_t cb,
-                                               float scale, bool mn, uint32_t mn_addr, uint32_t krow) {
+                                               float scale, uint8_t *mn_local, uint32_t mn_remote, uint32_t krow) {
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     float v[32];
@@ -139,7 +141,8 @@ __device__ __forceinline__ void pair_row_to_op(uint32_t src, uint32_t pk, uint8_
       const uint4 u = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
       const uint32_t c8 = 8u * cb + 4u * i + j;            // 16-byte chunk of the 256-column row
       if (kdst) *reinterpret_cast<uint4 *>(kdst + kmaj_off(r, c8)) = u;
-      if (mn) st_cluster_v4(mn_addr + mn_off(krow, c8 & 15u), u);
+      if (MN == kMnLocal) *reinterpret_cast<uint4 *>(mn_local + mn_off(krow, c8 & 15u)) = u;
+      if (MN == kMnRemote) st_cluster_v4(mn_remote + mn_off(krow, c8 & 15u), u);
     }
   }
   tmem_wait_st();
@@ -229,6 +232,27 @@ __device__ __forceinline__ void prefetch_rows(const CUtensorMap *m, const TileCo
     if (64 * j < t.w) tma_prefetch_l2_2d(m, t.x0 + 64 * j, t.y0 + 128 * static_cast<int>(c));
 }
 
+// 16 values of M' (row `row`, columns col .. col + 15 of a block) straight to
+// global memory: one 32-byte store where the address allows it, two 16-byte
+// stores otherwise, element stores at a ragged edge.
+__device__ __forceinline__ void store16_global(const DevBlock &b, int32_t row, int32_t col, const float *m) {
+  if (row >= b.rows || col >= b.cols) return;
+  __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(b.ptr[kRoleIn]) + static_cast<int64_t>(row) * b.ld[kRoleIn] + col;
+  if (col + 16 <= b.cols) {
+    const uint4 u0 = pack8_bf16(m), u1 = pack8_bf16(m + 8);
+    if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(u0.x), "r"(u0.y),
+                   "r"(u0.z), "r"(u0.w), "r"(u1.x), "r"(u1.y), "r"(u1.z), "r"(u1.w)
+                   : "memory");
+    } else {
+      reinterpret_cast<uint4 *>(dst)[0] = u0;
+      reinterpret_cast<uint4 *>(dst)[1] = u1;
+    }
+  } else {
+    for (int e = 0; e < 16 && col + e < b.cols; ++e) dst[e] = __float2bfloat16_rn(m[e]);
+  }
+}
+
 __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tmem) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t c = cluster_ctarank();           // 0: even CTA (issues the MMAs), 1: odd CTA
@@ -239,42 +263,65 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
   const uint32_t grow = 128u * c + r;             // row of the tile
   const uint32_t tP = tmem + ((q * 32) << 16);    // this warp's lanes of D_P (columns 0..255)
   const uint32_t tX = tP + 256u;                  // ... and of D_X (columns 256..511)
-  uint8_t *Xs = sm.x(), *Ss = sm.s();
+  uint8_t *Xs = sm.x(), *Ss = sm.s(), *Xmn = sm.mn();
   const bool step_mode = a.mode == 1;
   const bool has_w = step_mode && a.has_w;
   const bool leader = c == 0 && threadIdx.x == 0;
   const bool tma = threadIdx.x == 0;              // this CTA's TMA-issuing thread
-  // X_mn of the CTA that owns this thread's columns (itself or the partner)
-  const uint32_t mn_owner = cb >> 1;
-  const uint32_t mn_addr = mapa_shared(smem_u32(sm.mn()), mn_owner);
-  // the even CTA's ready barrier (local for c = 0)
+  // This warp's columns belong to X_mn of CTA cb / 2: its own or the partner's.
+  const bool mn_remote = (cb >> 1) != c;
+  const uint32_t mn_remote_addr = mapa_shared(smem_u32(Xmn), peer);
+  // the even CTA's ready barrier: its own warps arrive locally, the odd CTA's
+  // through the cluster (release at cluster scope)
   const uint32_t ready_addr = mapa_shared(smem_u32(sm.bar_ready()), 0);
   const uint32_t peer_norm_addr = mapa_shared(smem_u32(sm.peer_norm()), peer);
   const uint32_t peer_norm_bar = mapa_shared(smem_u32(sm.bar_norm()), peer);
   const int64_t n_pairs = gridDim.x / 2;
   const int64_t pair = blockIdx.x / 2;
+  const uint32_t ld_bytes = (step_mode ? 2u : 1u) * 4u * kChunk;
+  // The next tile's M (to X_s, after the last Gram product) and G (to X_mn,
+  // after the last update product) are loaded during the current tile's last
+  // step, unless X_s stages O for the epilogue.
+  const bool prefetch = !a.has_o;
   uint32_t it = 0, job = 0;
   uint32_t ld_armed = 0, ld_seen = 0, w_armed = 0, w_seen = 0, mma_issued = 0;
-  TileCoord *cur = sm.coord(0), *nxt = sm.coord(1);
+  bool ld_issued = false;   // (TMA thread) the current tile's loads are out
+  bool g_pending = false;   // (TMA thread) the next tile's M is out, its G not yet
+  // Tile coordinates alternate between two slots: the TMA thread decodes tile
+  // it + 1 into the other slot before it arms that tile's loads, so a thread
+  // that has seen the loads land also sees the coordinates.
   if (a.test_stall && pair == 0) pair_wait(sm.bar_never(), 0, sm, peer, a.status);
-  if (tma) *cur = decode_tile(a, nullptr, pair);
+  if (tma) *sm.coord(0) = decode_tile(a, nullptr, pair);
   __syncthreads();
   bool bad = *sm.abort_flag() != 0;
 
+  // this CTA's arrival on the ready barrier once its warp's operands are written
+  auto ready = [&]() {
+    __syncwarp();
+    if (lane == 0) {
+      if (c == 0) mbar_arrive(sm.bar_ready());
+      else mbar_arrive_cluster(ready_addr);
+    }
+  };
+
   for (int64_t tile = pair; tile < a.n_tiles && !bad; tile += n_pairs, ++it) {
-    if (tma) {
+    TileCoord *cur = sm.coord(it & 1u), *nxt = sm.coord((it + 1u) & 1u);
+    if (tma && !ld_issued) {
       bulk_wait_read0();   // the previous tile's stores have finished reading X_s / S_s
-      mbar_arrive_expect_tx(sm.bar_ld(), (step_mode ? 2u : 1u) * 4u * kChunk);
+      mbar_arrive_expect_tx(sm.bar_ld(), ld_bytes);
       load_rows(a.tmaps + cur->tm[kRoleIn], Xs, *cur, c, sm.bar_ld());
-      if (step_mode) load_rows(a.tmaps + cur->tm[kRoleG], Ss, *cur, c, sm.bar_ld());
+      if (step_mode) load_rows(a.tmaps + cur->tm[kRoleG], Xmn, *cur, c, sm.bar_ld());
       ++ld_armed;
     }
+    ld_issued = false;
     __syncwarp();
     bad = !pair_wait(sm.bar_ld(), it & 1u, sm, peer, a.status);
     if (tma && !bad) ++ld_seen;
     if (__any_sync(0xffffffffu, bad)) break;
 
-    // ---- prologue: M' = mu M + G (or the plain input), this CTA's ||.||_F^2, fp32 copy to D_X
+    // ---- prologue: M' = mu M + G (or the plain input) to HBM, this CTA's
+    // ||.||_F^2, fp32 copy to D_X.  M lands in X_s, G in X_mn (K-major boxes).
+    const DevBlock &blk = a.blocks[cur->blk];
     float sumsq = 0.f;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -286,10 +333,9 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
         unpack8(*reinterpret_cast<const uint4 *>(Xs + kmaj_off(r, c8)), m);
         if (step_mode) {
           float g[8];
-          unpack8(*reinterpret_cast<const uint4 *>(Ss + kmaj_off(r, c8)), g);
+          unpack8(*reinterpret_cast<const uint4 *>(Xmn + kmaj_off(r, c8)), g);
 #pragma unroll
           for (int e = 0; e < 8; ++e) m[e] = fmaf(a.mu, m[e], g[e]);
-          *reinterpret_cast<uint4 *>(Ss + kmaj_off(r, c8)) = pack8_bf16(m);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -297,12 +343,17 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
           sumsq = fmaf(m[e], m[e], sumsq);
         }
       }
+      if (step_mode) {   // M' of this row's 32 columns: 64 contiguous bytes
+        const int32_t row = cur->y0 + static_cast<int32_t>(grow);
+        const int32_t col = cur->x0 + static_cast<int32_t>(64 * cb + 32 * i);
+        store16_global(blk, row, col, v);
+        store16_global(blk, row, col + 16, v + 16);
+      }
       tmem_st32(tX + 64 * cb + 32 * i, v);
     }
     tmem_wait_st();
     sumsq = warp_sum(sumsq);
     if (lane == 0) sm.red()[warp] = sumsq;
-    if (step_mode) fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.bar_pro());
@@ -313,10 +364,6 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) own += sm.red()[w];
     if (tma) {
-      if (step_mode) {
-        store_rows(a.tmaps + cur->tm[kRoleIn], Ss, *cur, c);
-        bulk_commit();
-      }
       st_cluster_f32(peer_norm_addr, own);   // the partner's half of the tile norm
       mbar_arrive_cluster(peer_norm_bar);
     }
@@ -331,15 +378,22 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
       f16 = min(cur->h, cur->w) <= 64 && !(total > 0.f && nrm < kTinyNorm * rho);
 
     // ---- operand g_0 X_0 = r(g_0 M' / rho): X_s, packed in D_X, and X_mn of the column owner
-    if (f16) pair_row_to_op<0>(tX, tX, Xs, r, cb, a.gamma0 / rho, true, mn_addr, grow);
-    else pair_row_to_op<1>(tX, tX, Xs, r, cb, a.gamma0 / rho, true, mn_addr, grow);
-    // M' must have left S_s before the first conversion (after MMA1) overwrites
-    // it: MMA1 waits for this thread's arrival below
-    if (step_mode && tma) bulk_wait_read0();
-    fence_proxy_async_cluster();
+    // (X_s and X_mn were read by every thread of this CTA before bar_pro, and
+    // the partner wrote its norm only after its own bar_pro)
+    if (mn_remote) {
+      if (f16) pair_row_to_op<0, kMnRemote>(tX, tX, Xs, r, cb, a.gamma0 / rho, Xmn, mn_remote_addr, grow);
+      else pair_row_to_op<1, kMnRemote>(tX, tX, Xs, r, cb, a.gamma0 / rho, Xmn, mn_remote_addr, grow);
+      fence_proxy_async_cluster();
+    } else {
+      if (f16) pair_row_to_op<0, kMnLocal>(tX, tX, Xs, r, cb, a.gamma0 / rho, Xmn, mn_remote_addr, grow);
+      else pair_row_to_op<1, kMnLocal>(tX, tX, Xs, r, cb, a.gamma0 / rho, Xmn, mn_remote_addr, grow);
+      fence_proxy_async_smem();
+    }
+    // the previous tile's W' (and O) stores must have left S_s / X_s before
+    // MMA1 completes and the first conversion overwrites S_s
+    if (tma) bulk_wait_read0();
     tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(ready_addr);
+    ready();
     if (leader) {
       bad = !pair_wait(sm.bar_ready(), job & 1u, sm, peer, a.status);
       if (!bad) {
@@ -360,16 +414,23 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
     bool stop = false;
     for (int t = 0; t < a.K && !stop; ++t) {
       const ResidentStep *stp = &a.step[t];
+      const bool last = t + 1 == a.K;
       // after MMA1: S = r(s D_P) to S_s and (packed) to D_X
       bad = !pair_wait(sm.bar_mma(), job++ & 1u, sm, peer, a.status);
       if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
-      if (f16) pair_row_to_op<0>(tP, tX, Ss, r, cb, stp->s, false, 0, 0);
-      else pair_row_to_op<1>(tP, tX, Ss, r, cb, stp->s, false, 0, 0);
+      if (last && prefetch && tma && nxt->blk >= 0) {   // X_s is free: the next tile's M
+        mbar_arrive_expect_tx(sm.bar_ld(), ld_bytes);
+        load_rows(a.tmaps + nxt->tm[kRoleIn], Xs, *nxt, c, sm.bar_ld());
+        ++ld_armed;
+        g_pending = step_mode;
+        ld_issued = true;
+      }
+      if (f16) pair_row_to_op<0, kMnNone>(tP, tX, Ss, r, cb, stp->s, nullptr, 0, 0);
+      else pair_row_to_op<1, kMnNone>(tP, tX, Ss, r, cb, stp->s, nullptr, 0, 0);
       fence_proxy_async_smem();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(ready_addr);
+      ready();
       if (leader) {
         bad = !pair_wait(sm.bar_ready(), job & 1u, sm, peer, a.status);
         if (!bad) {
@@ -382,7 +443,7 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
       bad = !pair_wait(sm.bar_mma(), job++ & 1u, sm, peer, a.status);
       if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
-      if (t + 1 == a.K && has_w && tma) {   // S_s is free for good: W lands there for the epilogue
+      if (last && has_w && tma) {   // S_s is free for good: W lands there for the epilogue
         mbar_arrive_expect_tx(sm.bar_w(), 4u * kChunk);
         load_rows(a.tmaps + cur->tm[kRoleW], Ss, *cur, c, sm.bar_w());
         ++w_armed;
@@ -390,8 +451,7 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
       if (f16) pair_row_to_bop<0>(tP, grow, cb, stp->beta, stp->a);
       else pair_row_to_bop<1>(tP, grow, cb, stp->beta, stp->a);
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(ready_addr);
+      ready();
       if (leader) {
         bad = !pair_wait(sm.bar_ready(), job & 1u, sm, peer, a.status);
         if (!bad) {
@@ -404,13 +464,18 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
       bad = !pair_wait(sm.bar_mma(), job++ & 1u, sm, peer, a.status);
       if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
-      if (t + 1 < a.K) {
-        if (f16) pair_row_to_op<0>(tX, tX, Xs, r, cb, stp->xr, true, mn_addr, grow);
-        else pair_row_to_op<1>(tX, tX, Xs, r, cb, stp->xr, true, mn_addr, grow);
-        fence_proxy_async_cluster();
+      if (!last) {
+        if (mn_remote) {
+          if (f16) pair_row_to_op<0, kMnRemote>(tX, tX, Xs, r, cb, stp->xr, Xmn, mn_remote_addr, grow);
+          else pair_row_to_op<1, kMnRemote>(tX, tX, Xs, r, cb, stp->xr, Xmn, mn_remote_addr, grow);
+          fence_proxy_async_cluster();
+        } else {
+          if (f16) pair_row_to_op<0, kMnLocal>(tX, tX, Xs, r, cb, stp->xr, Xmn, mn_remote_addr, grow);
+          else pair_row_to_op<1, kMnLocal>(tX, tX, Xs, r, cb, stp->xr, Xmn, mn_remote_addr, grow);
+          fence_proxy_async_smem();
+        }
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ready_addr);
+        ready();
         if (leader) {
           bad = !pair_wait(sm.bar_ready(), job & 1u, sm, peer, a.status);
           if (!bad) {
@@ -419,6 +484,9 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
           }
         }
         if ((stop = __any_sync(0xffffffffu, bad))) break;
+      } else if (prefetch && step_mode && tma && nxt->blk >= 0) {   // X_mn is free: the next tile's G
+        load_rows(a.tmaps + nxt->tm[kRoleG], Xmn, *nxt, c, sm.bar_ld());
+        g_pending = false;
       }
     }
     if (stop) break;
@@ -465,14 +533,17 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
         if (has_w) store_rows(a.tmaps + cur->tm[kRoleW], Ss, *cur, c);
         bulk_commit();
       }
-      *cur = *nxt;
     }
-    // The next tile's loads (issued by the TMA thread after its stores have
-    // read X_s / S_s) gate everyone's next prologue.
     if (__any_sync(0xffffffffu, bad)) break;
   }
   if (tma) {
-    // After an abort: wait (bounded) for this CTA's loads still in flight.
+    // After an abort: wait (bounded) for this CTA's loads still in flight.  A
+    // prefetched M whose G was not issued yet gets its G now, so that the
+    // phase armed for both completes (X_mn's content no longer matters).
+    if (g_pending) {   // the loop left tile `it` early: its successor's slot
+      const TileCoord &nx = *sm.coord((it + 1u) & 1u);
+      load_rows(a.tmaps + nx.tm[kRoleG], Xmn, nx, c, sm.bar_ld());
+    }
     for (; ld_seen < ld_armed; ++ld_seen) mbar_wait(sm.bar_ld(), ld_seen & 1u, a.status);
     for (; w_seen < w_armed; ++w_seen) mbar_wait(sm.bar_w(), w_seen & 1u, a.status);
     bulk_wait0();
