@@ -458,7 +458,7 @@ __device__ void pair_main(const ResidentArgs &a, const PairSmem &sm, uint32_t tm
     bad = !send_stage();
     if (leader && !bad) bad = !issue(kJobGram, nullptr, false);
     if (tma) {   // next tile of this pair, while MMA1 runs
-      *nxt = decode_tile(a, nullptr, tile + n_pairs);
+      *nxt = decode_tile(a, nullptr, tile + n_pairs, cur->blk);
       if (nxt->blk >= 0) {
         prefetch_rows(a.tmaps + nxt->tm[kRoleIn], *nxt, c);
         if (step_mode) prefetch_rows(a.tmaps + nxt->tm[kRoleG], *nxt, c);

@@ -121,6 +121,17 @@ static __device__ __noinline__ TileCoord decode_tile(const ResidentArgs &a, cons
     for (int r = 0; r < kNumRoles; ++r) t.tm[r] = b.tm[r];
     return t;
   }
+  if (hint >= 0) {  // a later tile than one in block `hint`: that block or one after it, usually
+                    // the same or the next (one or two dependent loads instead of a full search)
+    lo = hint;
+    for (int k = 0; k < 2 && lo < hi; ++k) {
+      if (a.blocks[lo + 1].tile_begin > tile) {
+        hi = lo;
+        break;
+      }
+      ++lo;
+    }
+  }
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (a.blocks[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
