@@ -489,7 +489,9 @@ def run_ours(args):
     prof = load_profile_traffic(T) if tiles is None else None
     roofline = {
         "bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved / peak_burst,
-        "traffic": prof, "kernel": "ns_resident_kernel" if tiles is None else "whole step (on-chip and staged launches)",
+        "traffic": prof,
+        "kernel": (ONCHIP_KERNELS.get(T, "staged") + "_kernel" if tiles is None
+                   else "whole step (on-chip and staged launches)"),
         "peak_source": f"bf16_tflops, burst ({peak_src})",
         "frac_sustained": achieved / peak_sus, "peak_sustained": peak_sus,
         "frac_sym": sym_flops / (ms_step / 1e3) / 1e12 / peak_burst,
@@ -532,17 +534,31 @@ def run_ours(args):
     return 0
 
 
+ONCHIP_KERNELS = {128: "ns_resident", 256: "ns_pair"}   # the on-chip kernel of each tile edge
+KERNEL_HEADERS = ("onchip.cuh", "ptx.cuh")
+
+
+def kernel_source_sha(kernel: str) -> str:
+    """sha256 prefix of an on-chip kernel's source and the device headers it shares."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in (kernel + ".cu",) + KERNEL_HEADERS:
+        with open(os.path.join(ROOT, "tiled_newton_schulz_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def load_profile_traffic(T: int):
     """DRAM bytes per launch of the on-chip kernel from the committed ncu
     summary, or None when there is none or the kernel source changed since."""
-    import hashlib
-    p = os.path.join(ROOT, "profiles", f"ns_resident_llama7b_T{T}_traffic.json")
-    src = os.path.join(ROOT, "tiled_newton_schulz_b200", "csrc", "ns_resident.cu")
+    kernel = ONCHIP_KERNELS.get(T)
+    if kernel is None:
+        return None
+    p = os.path.join(ROOT, "profiles", f"{kernel}_llama7b_T{T}_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        sha = kernel_source_sha(kernel)
     except OSError:
         return None
     return d.get("dram_bytes_per_full_launch") if d.get("kernel_source_sha256_prefix") == sha else None
