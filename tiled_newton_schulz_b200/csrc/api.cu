@@ -585,6 +585,9 @@ Epilogue epi(float alpha, float beta, const float *c32, float *out32, void *out1
   e.out16 = out16;
   e.out16_dtype = dt;
   e.diag = 0.f;
+  e.out2_32 = nullptr;
+  e.out2_16 = nullptr;
+  e.diag2 = 0.f;
   e.sym = 0;
   return e;
 }
@@ -637,7 +640,7 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       na.x16_dtype = dt16;
       na.partial = pk.partial;
       na.parts = pk.parts;
-      na.keep32 = (f32 || gram) ? 1 : 0;   // the 16-bit NS path reads only the 16-bit copy
+      na.keep32 = f32 ? 1 : 0;   // the 16-bit paths (NS and Gram NS) read only the 16-bit copy
       na.eps = p.eps;
       na.safety = safety;
       HIMUON_TRY(launch_normalize(na, stream));
@@ -714,7 +717,8 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
                 cur = 1 - cur;
                 xfinal = x32[cur];
               } else {
-                rc = ops.mm(qop(qc), n, n, x16[cur], n, m, 0, n, m, n, bc, epi(1.f, 0.f, nullptr, x32[0], x16[1 - cur], dt16));
+                // (the fp32 copy of X is written by the final product only)
+                rc = ops.mm(qop(qc), n, n, x16[cur], n, m, 0, n, m, n, bc, epi(1.f, 0.f, nullptr, nullptr, x16[1 - cur], dt16));
                 cur = 1 - cur;
               }
               if (rc) break;
@@ -723,14 +727,18 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
             }
             q_identity = true;
           }
-          // Z = b R + c R^2 (its fp32 copy feeds only Q = Z + aI right after Q = I,
-          // or every product when the operands are fp32)
-          rc = ops.mm(rop(), n, n, rop(), n, n, 0, n, n, n, bc,
-                      sym(epi(cc, b, r32, (f32 || q_identity) ? z32 : nullptr, z16, dt16)));
+          // Z = b R + c R^2 (fp32 copy only when the operands are fp32).  Right
+          // after Q = I the same epilogue also writes Q <- Q Z + a Q = Z + a I.
+          Epilogue ez = sym(epi(cc, b, r32, f32 ? z32 : nullptr, z16, dt16));
+          if (q_identity) {
+            ez.out2_32 = qf[qc];
+            ez.out2_16 = f32 ? nullptr : q16[qc];
+            ez.diag2 = a;
+          }
+          rc = ops.mm(rop(), n, n, rop(), n, n, 0, n, n, n, bc, ez);
           if (rc) break;
           // Q <- Q Z + a Q
           if (q_identity) {
-            HIMUON_TRY(launch_add_identity(z32, a, qf[qc], f32 ? nullptr : q16[qc], dt16, n, bc, stream));
             q_identity = false;
           } else {
             rc = ops.mm(qop(qc), n, n, zop(), n, n, 0, n, n, n, bc,

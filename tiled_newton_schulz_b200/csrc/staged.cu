@@ -151,16 +151,43 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
   if (threadIdx.x == 0) a.partial[t * a.parts + blockIdx.x] = s;
 }
 
-// grid (chunks, tiles): rho from the partial sums (fixed order), then scale.
+// grid (chunks, tiles): rho from the partial sums (fixed order), then scale,
+// four elements per access (16-byte fp32 loads and stores, 8-byte 16-bit
+// stores; a tile's chunk starts at a multiple of 8 elements).
 __global__ void __launch_bounds__(256) normalize_kernel(const NormArgs a) {
   const int64_t t = blockIdx.y;
   float s = 0.f;
   for (int p = 0; p < a.parts; ++p) s += a.partial[t * a.parts + p];
   const float inv = 1.0f / ((sqrtf(s) + a.eps) * a.safety);
   float *x = a.x32 + t * a.elems;
-  const int64_t per = (a.elems + gridDim.x - 1) / gridDim.x;
+  const int64_t per = ((a.elems + gridDim.x - 1) / gridDim.x + 7) / 8 * 8;
   const int64_t e0 = blockIdx.x * per, e1 = min(a.elems, e0 + per);
-  for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+  // (the planner pads tiles to multiples of 128 rows and columns; any other
+  // size takes the element loop below)
+  const bool vec = (a.elems & 7) == 0;
+  int64_t e = vec ? e0 + 4 * threadIdx.x : e0 + threadIdx.x;
+  for (; vec && e + 4 <= e1; e += 4 * blockDim.x) {
+    float4 v = *reinterpret_cast<const float4 *>(x + e);
+    v.x *= inv;
+    v.y *= inv;
+    v.z *= inv;
+    v.w *= inv;
+    if (a.keep32) *reinterpret_cast<float4 *>(x + e) = v;
+    if (a.x16) {
+      uint2 u;
+      if (a.x16_dtype == HIMUON_FP16) {
+        __half2 *h = reinterpret_cast<__half2 *>(&u);
+        h[0] = __floats2half2_rn(v.x, v.y);
+        h[1] = __floats2half2_rn(v.z, v.w);
+      } else {
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+        h[0] = __floats2bfloat162_rn(v.x, v.y);
+        h[1] = __floats2bfloat162_rn(v.z, v.w);
+      }
+      *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(a.x16) + t * a.elems + e) = u;
+    }
+  }
+  for (; e < e1; e += vec ? 1 : blockDim.x) {   // element by element when not vectorised
     const float v = x[e] * inv;
     if (a.keep32) x[e] = v;
     if (a.x16) st_elem(a.x16, a.x16_dtype, t * a.elems + e, v);
@@ -218,16 +245,6 @@ __global__ void __launch_bounds__(256) unpack_kernel(const UnpackArgs a, int32_t
   }
 }
 
-__global__ void add_identity_kernel(const float *z, float a, float *q32, void *q16, int32_t dt, int64_t n,
-                                    int64_t total) {
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = (e / n) % n, c = e % n;
-    const float v = z[e] + (r == c ? a : 0.f);
-    q32[e] = v;
-    if (q16) st_elem(q16, dt, e, v);
-  }
-}
-
 // ---------------------------------------------------------------- epilogue
 struct EpiArgs {
   float alpha, beta, diag;
@@ -235,10 +252,47 @@ struct EpiArgs {
   float *out32;
   void *out16;
   int32_t out16_dtype;
+  float *out2_32;   // the same values + diag2 on the diagonal (nullptr: none)
+  void *out2_16;
+  float diag2;
   int32_t sym;      // lower-triangle tiles only, off-diagonal ones mirrored
   int64_t N;        // columns of the output matrices
   int64_t stride;   // elements per output matrix (M * N)
 };
+
+// Store 8 values v at element index `o` of an fp32 and/or a 16-bit output
+// (and mirrored, see epi_store8).
+__device__ __forceinline__ void epi_put8(const EpiArgs &e, float *out32, void *out16, int64_t o, const float *v,
+                                         bool mirror, int64_t om) {
+  if (out32) {
+    *reinterpret_cast<float4 *>(out32 + o) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(out32 + o + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    if (mirror) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out32[om + i * e.N] = v[i];
+    }
+  }
+  if (out16) {
+    uint4 u;
+    if (e.out16_dtype == HIMUON_FP16) {
+      __half2 *h = reinterpret_cast<__half2 *>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+      *reinterpret_cast<uint4 *>(static_cast<__half *>(out16) + o) = u;
+    } else {
+      __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out16) + o) = u;
+    }
+    if (mirror) {
+      const uint16_t *hs = reinterpret_cast<const uint16_t *>(&u);
+      uint16_t *d = static_cast<uint16_t *>(out16);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[om + i * e.N] = hs[i];
+    }
+  }
+}
 
 // Write 8 consecutive outputs starting at element index `o` of the batch;
 // they sit in row `row`, columns col..col+7 of their matrix.  With `mirror`
@@ -258,37 +312,18 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = e.alpha * acc[i];
   }
-  if (e.diag != 0.f && row >= col && row < col + 8) {
+  const bool on_diag = row >= col && row < col + 8;
+  if (e.diag != 0.f && on_diag) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] += (col + i == row) ? e.diag : 0.f;
   }
-  if (e.out32) {
-    *reinterpret_cast<float4 *>(e.out32 + o) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4 *>(e.out32 + o + 4) = make_float4(v[4], v[5], v[6], v[7]);
-    if (mirror) {
+  epi_put8(e, e.out32, e.out16, o, v, mirror, om);
+  if (e.out2_32 || e.out2_16) {
+    if (on_diag) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) e.out32[om + i * e.N] = v[i];
+      for (int i = 0; i < 8; ++i) v[i] += (col + i == row) ? e.diag2 : 0.f;
     }
-  }
-  if (e.out16) {
-    uint4 u;
-    if (e.out16_dtype == HIMUON_FP16) {
-      __half2 *h = reinterpret_cast<__half2 *>(&u);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
-      *reinterpret_cast<uint4 *>(static_cast<__half *>(e.out16) + o) = u;
-    } else {
-      __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-      *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(e.out16) + o) = u;
-    }
-    if (mirror) {
-      const uint16_t *hs = reinterpret_cast<const uint16_t *>(&u);
-      uint16_t *d = static_cast<uint16_t *>(e.out16);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) d[om + i * e.N] = hs[i];
-    }
+    epi_put8(e, e.out2_32, e.out2_16, o, v, mirror, om);
   }
 }
 
@@ -468,9 +503,13 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const float *A, const fl
     for (int j = 0; j < 4; ++j) {
       float v = ep.alpha * acc[i][j];
       if (ep.c32) v = fmaf(ep.beta, ep.c32[o + j], v);
-      if (m0 + ty * 4 + i == n0 + tx * 4 + j) v += ep.diag;
+      const bool d = m0 + ty * 4 + i == n0 + tx * 4 + j;
+      if (d) v += ep.diag;
       if (ep.out32) ep.out32[o + j] = v;
       if (ep.out16) st_elem(ep.out16, ep.out16_dtype, o + j, v);
+      if (d) v += ep.diag2;
+      if (ep.out2_32) ep.out2_32[o + j] = v;
+      if (ep.out2_16) st_elem(ep.out2_16, ep.out16_dtype, o + j, v);
     }
   }
 }
@@ -516,6 +555,9 @@ EpiArgs to_epi(const Epilogue &e, int64_t M, int64_t N) {
   a.out32 = e.out32;
   a.out16 = e.out16;
   a.out16_dtype = e.out16_dtype;
+  a.out2_32 = e.out2_32;
+  a.out2_16 = e.out2_16;
+  a.diag2 = e.diag2;
   a.sym = e.sym && M == N;
   a.N = N;
   a.stride = M * N;
@@ -593,15 +635,6 @@ cudaError_t launch_unpack(const UnpackArgs &a, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(parts), static_cast<unsigned>(a.n_tiles));
   count_launch();
   unpack_kernel<<<grid, 256, 0, stream>>>(a, static_cast<int32_t>(parts));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_add_identity(const float *z32, float a, float *q32, void *q16, int32_t q16_dtype, int64_t n,
-                                int64_t batch, cudaStream_t stream) {
-  const int64_t total = n * n * batch;
-  const int blocks = static_cast<int>((total + 255) / 256 < 65535 ? (total + 255) / 256 : 65535);
-  count_launch();
-  add_identity_kernel<<<blocks, 256, 0, stream>>>(z32, a, q32, q16, q16_dtype, n, total);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,11 @@ struct Epilogue {
   float *out32;
   void *out16;
   int32_t out16_dtype;
+  // A second output, the same values plus diag2 on the diagonal (e.g. Q = Z + a I
+  // beside Z); out2_16 has out16_dtype.
+  float *out2_32;
+  void *out2_16;
+  float diag2;
   // The product is symmetric (M == N; and c32, if given, symmetric): the
   // tensor-core version computes only the 128 x 128 tiles on and below the
   // diagonal and writes each off-diagonal one twice, mirrored.
@@ -79,9 +84,5 @@ struct UnpackArgs {
   float lr;
 };
 cudaError_t launch_unpack(const UnpackArgs &a, cudaStream_t stream);
-
-// q32/q16 <- z32 + a I  (n x n per matrix); used when Q = I in Gram NS
-cudaError_t launch_add_identity(const float *z32, float a, float *q32, void *q16, int32_t q16_dtype, int64_t n,
-                                int64_t batch, cudaStream_t stream);
 
 }  // namespace himuon
