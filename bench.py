@@ -77,9 +77,10 @@ def workload_tiles(shapes_splits, T, sym=False):
     for (H, W), split in shapes_splits:
         blocks = [(H, W)] if split is None else [((H, s) if split[0] == 1 else (s, W)) for s in split[1]]
         for (h, w) in blocks:
-            for r0 in range(0, h, T):
-                for c0 in range(0, w, T):
-                    th, tw = min(T, h - r0), min(T, w - c0)
+            Tb = T if T > 0 else max(h, w)   # T <= 0: the whole block is one tile
+            for r0 in range(0, h, Tb):
+                for c0 in range(0, w, Tb):
+                    th, tw = min(Tb, h - r0), min(Tb, w - c0)
                     tiles += 1
                     flops += (sym_flops_per_tile if sym else flops_per_tile)(th, tw, K_STEPS)
     return tiles, flops
@@ -490,8 +491,8 @@ def run_ours(args):
     roofline = {
         "bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved / peak_burst,
         "traffic": prof,
-        "kernel": (ONCHIP_KERNELS.get(T, "staged") + "_kernel" if tiles is None
-                   else "whole step (on-chip and staged launches)"),
+        "kernel": ((ONCHIP_KERNELS[T] + "_kernel" if T in ONCHIP_KERNELS else "gemm_tc_kernel (staged path)")
+                   if tiles is None else "whole step (on-chip and staged launches)"),
         "peak_source": f"bf16_tflops, burst ({peak_src})",
         "frac_sustained": achieved / peak_sus, "peak_sustained": peak_sus,
         "frac_sym": sym_flops / (ms_step / 1e3) / 1e12 / peak_burst,

@@ -328,11 +328,18 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
 }
 
 // ---------------------------------------------------------------- tcgen05 GEMM
-// Pipeline depth: 3 stages for long K; 2 when K <= 256 (at most 4 k-blocks),
-// which lets 3 CTAs share an SM and hide each other's latency.
-constexpr uint32_t kStageA = 16384, kStageB = 16384, kStageBytes = kStageA + kStageB;
-template <int STAGES>
-constexpr uint32_t gemm_smem() { return STAGES * kStageBytes + 128 + 1024; }
+// A CTA computes a 128 x BN output tile (BN = 128, or 256 for products that
+// are not symmetric and have N a multiple of 256: a 128 x 256 x 16 MMA reads
+// 12 KB of operands from shared memory in 128 cycles where two 128 x 128 x 16
+// ones read 16 KB, which keeps the operand traffic under the shared-memory
+// bandwidth).  Pipeline depth for 128-column tiles: 3 stages for long K; 2
+// when K <= 256 (at most 4 k-blocks), which lets more CTAs share an SM and
+// hide each other's latency; 256-column tiles always take 2.
+constexpr uint32_t kStageA = 16384;
+template <int BN>
+__host__ __device__ constexpr uint32_t stage_bytes() { return kStageA + BN * 128u; }
+template <int STAGES, int BN>
+constexpr uint32_t gemm_smem() { return STAGES * stage_bytes<BN>() + 128 + 1024; }
 constexpr int kGemmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 
 struct GemmTcArgs {
@@ -342,10 +349,11 @@ struct GemmTcArgs {
   int *status;
 };
 
-template <int B_MN, int kStages>
+template <int B_MN, int kStages, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                    const GemmTcArgs a) {
+  constexpr uint32_t kStageBytes = stage_bytes<BN>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + kStages * kStageBytes);
@@ -353,7 +361,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *done = empty + kStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t n0 = blockIdx.x * 128, m0 = blockIdx.y * 128;
+  int32_t n0 = blockIdx.x * BN, m0 = blockIdx.y * 128;
   const int32_t z = blockIdx.z;
   if (a.ep.sym) {   // blockIdx.x enumerates the tiles (ti, tj), tj <= ti, row by row
     const int32_t k = blockIdx.x;
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int64_t per = G * gx, g = L / per, r = L % per;
     const int64_t gm = (gy - g * G) < G ? (gy - g * G) : G;
     m0 = static_cast<int32_t>((g * G + r % gm) * 128);
-    n0 = static_cast<int32_t>((r / gm) * 128);
+    n0 = static_cast<int32_t>((r / gm) * BN);
   }
   const bool mirror = a.ep.sym && m0 != n0;
   const int nk = static_cast<int>(a.K / 64);
@@ -389,7 +397,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&mapB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -404,10 +412,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint8_t *As = sm + s * kStageBytes, *Bs = As + kStageA;
       mbar_arrive_expect_tx(full + s, kStageBytes);
       tma_load_3d(As, &mapA, kb * 64, m0, z, full + s);
-      if (B_MN) {
-        tma_load_3d(Bs, &mapB, n0, kb * 64, z, full + s);
-        tma_load_3d(Bs + 8192, &mapB, n0 + 64, kb * 64, z, full + s);
-      } else {
+      if (B_MN) {   // BN / 64 boxes of 64 columns x 64 k-rows
+#pragma unroll
+        for (int j = 0; j < BN / 64; ++j) tma_load_3d(Bs + 8192 * j, &mapB, n0 + 64 * j, kb * 64, z, full + s);
+      } else {      // one box of 64 k-columns x BN rows
         tma_load_3d(Bs, &mapB, kb * 64, n0, z, full + s);
       }
     }
@@ -434,8 +442,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
       const int64_t obase = z * a.ep.stride + static_cast<int64_t>(m0 + row) * a.ep.N + n0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
+#pragma unroll 1
+      for (int i = 0; i < BN / 32; ++i) {
         float v[32];
         tmem_ld32(taddr + 32 * i, v);
         tmem_wait_ld();
@@ -453,7 +461,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, BN);
   }
 }
 
@@ -569,19 +577,20 @@ EpiArgs to_epi(const Epilogue &e, int64_t M, int64_t N) {
 cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int64_t N, int64_t K, int64_t batch,
                     const Epilogue &ep, int *status, cudaStream_t stream) {
   if (M % 128 || N % 128 || K % 64 || batch < 1 || batch > 65535) return cudaErrorInvalidValue;
+  GemmTcArgs a;
+  a.K = K;
+  a.ep = to_epi(ep, M, N);
+  a.status = status;
+  const int BN = (!a.ep.sym && N % 256 == 0) ? 256 : 128;
   CUtensorMap ma, mb;
   if (!make_batch_map(&ma, A, batch, 64, 128)) return cudaErrorInvalidValue;
   if (b_trans) {
-    if (!make_batch_map(&mb, B, batch, 64, 128)) return cudaErrorInvalidValue;
+    if (!make_batch_map(&mb, B, batch, 64, static_cast<uint32_t>(BN))) return cudaErrorInvalidValue;
   } else {
     if (!make_batch_map(&mb, B, batch, 64, 64)) return cudaErrorInvalidValue;
   }
-  GemmTcArgs a;
-  a.K = K;
-  a.idesc = idesc_f16(128, 128, A.dtype == HIMUON_FP16 ? 0u : 1u, 0, b_trans ? 0u : 1u, 0);
-  a.ep = to_epi(ep, M, N);
-  a.status = status;
-  dim3 grid(static_cast<unsigned>(N / 128), static_cast<unsigned>(M / 128), static_cast<unsigned>(batch));
+  a.idesc = idesc_f16(128, static_cast<uint32_t>(BN), A.dtype == HIMUON_FP16 ? 0u : 1u, 0, b_trans ? 0u : 1u, 0);
+  dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(M / 128), static_cast<unsigned>(batch));
   if (a.ep.sym) {
     const int64_t nt = M / 128;
     grid = dim3(static_cast<unsigned>(nt * (nt + 1) / 2), 1, static_cast<unsigned>(batch));
@@ -595,8 +604,15 @@ cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int6
     return cudaSuccess;
   };
   const bool short_k = K <= 256;
-  if (b_trans) e = short_k ? go(gemm_tc_kernel<0, 2>, gemm_smem<2>()) : go(gemm_tc_kernel<0, 3>, gemm_smem<3>());
-  else e = short_k ? go(gemm_tc_kernel<1, 2>, gemm_smem<2>()) : go(gemm_tc_kernel<1, 3>, gemm_smem<3>());
+  if (BN == 256) {
+    // two stages (97 KB): two CTAs share an SM, so one's epilogue overlaps the
+    // other's main loop (three stages, one CTA per SM, ran 6% slower)
+    if (b_trans) e = go(gemm_tc_kernel<0, 2, 256>, gemm_smem<2, 256>());
+    else e = go(gemm_tc_kernel<1, 2, 256>, gemm_smem<2, 256>());
+  } else {
+    if (b_trans) e = short_k ? go(gemm_tc_kernel<0, 2, 128>, gemm_smem<2, 128>()) : go(gemm_tc_kernel<0, 3, 128>, gemm_smem<3, 128>());
+    else e = short_k ? go(gemm_tc_kernel<1, 2, 128>, gemm_smem<2, 128>()) : go(gemm_tc_kernel<1, 3, 128>, gemm_smem<3, 128>());
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
