@@ -445,7 +445,7 @@ def _loop_reference(T, mode):
 
 
 @pytest.mark.parametrize("mode", ["ns", "step", "step_out"])
-@pytest.mark.parametrize("T,ctas", [(256, 2), (256, 6), (128, 1), (128, 3)])
+@pytest.mark.parametrize("T,ctas", [(256, 2), (256, 6), (128, 1), (128, 3), (64, 1), (64, 3), (32, 2)])
 def test_onchip_tile_loop(hm, monkeypatch, T, ctas, mode):
     """HIMUON_MAX_CTAS caps the launch so that every CTA (pair) runs many
     tiles of three matrices in its loop: tile coordinates, loads issued

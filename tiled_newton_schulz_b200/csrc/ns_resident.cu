@@ -182,6 +182,73 @@ __device__ __forceinline__ void tmem_row_to_tmem_op(uint32_t taddr, uint32_t r, 
   tmem_wait_st();
 }
 
+// ---- stacked super-tiles of two 64 x 64 tiles (P = 2)
+// The tiles sit on top of each other as rows 64 j .. 64 j + 63 of a 128 x 64
+// operand (the TMA staging layout already is that: one 128-byte swizzled
+// block).  The warp of half hf of a row covers its columns 32 hf .. 32 hf + 31.
+// v (those 32 fp32 values) -> r(scale v): packed to TMEM columns
+// pa + 16 hf .. pa + 16 hf + 15 (K values 32 hf .. 32 hf + 31 of the A
+// operand) and K-major to row r of `dst`.
+template <int F, bool SCALE>
+__device__ __forceinline__ void stack_row_to_op(const float (&v)[32], uint32_t pa, uint8_t *dst, uint32_t r,
+                                                uint32_t hf, float scale) {
+  uint32_t p[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    p[e] = SCALE ? pack2_op<F>(v[2 * e] * scale, v[2 * e + 1] * scale) : pack2_op<F>(v[2 * e], v[2 * e + 1]);
+  tmem_st16(pa + 16u * hf, p);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4 *>(dst + sw128_off(r, 4u * hf + j)) = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+  tmem_wait_st();
+}
+template <int F, bool SCALE>
+__device__ __forceinline__ void stack_tmem_to_op(uint32_t src, uint32_t pa, uint8_t *dst, uint32_t r, uint32_t hf,
+                                                 float scale) {
+  float v[32];
+  tmem_ld32(src, v);
+  tmem_wait_ld();
+  stack_row_to_op<F, SCALE>(v, pa, dst, r, hf, scale);
+}
+// The block-diagonal A operand of the update, Bop = r(beta D_P + diag I) on
+// row r's tile (tile r / 64, whose K values are packed at columns
+// 32 (r / 64) .. + 31) and zeros on the other tile's K values.  The warp of
+// half hf writes packed columns pa + 32 hf .. + 31: the Bop values when they
+// are its row's tile's (read from D_P columns 64 (r / 64) .. + 63), else zeros.
+template <int F>
+__device__ __forceinline__ void stack_row_to_bop(uint32_t tp, uint32_t pa, uint32_t r, uint32_t hf, float beta,
+                                                 float diag) {
+  const uint32_t jr = r >> 6;            // the same in the whole warp
+  uint32_t p[16];
+  if (hf == jr) {
+    const uint32_t lane = r & 31u, dchunk = (r >> 5) & 1u;   // diagonal: chunk (r % 64) / 32, position r % 32
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float v[32];
+      tmem_ld32(tp + 64u * jr + 32u * i, v);
+      tmem_wait_ld();
+      if (dchunk == static_cast<uint32_t>(i)) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a0 = fmaf(beta, v[2 * e], lane == 2u * e ? diag : 0.f);
+          const float a1 = fmaf(beta, v[2 * e + 1], lane == 2u * e + 1u ? diag : 0.f);
+          p[e] = pack2_op<F>(a0, a1);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) p[e] = pack2_op<F>(beta * v[2 * e], beta * v[2 * e + 1]);
+      }
+      tmem_st16(pa + 32u * hf + 16u * i, p);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) p[e] = 0u;
+    tmem_st16(pa + 32u * hf, p);
+    tmem_st16(pa + 32u * hf + 16u, p);
+  }
+  tmem_wait_st();
+}
+
 __device__ __forceinline__ bool use_smem_blocks(const ResidentArgs &a) {
   return a.smem_blocks != 0 && a.n_blocks <= kMaxSmemBlocks;
 }
@@ -284,7 +351,7 @@ enum Job { kJobGram = 0, kJobSquare = 1, kJobUpdate = 2 };
 // All threads of the group have written (and fenced) the operands of `job`:
 // one thread issues its eight 128x128x16 MMAs and commits them to bar_mma.
 // f16: the operands are fp16 (else bf16).
-template <int JOB>
+template <int JOB, int P>
 __device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st, bool f16);
 
 // A warp of group g has written (and fenced) its share of the operands of
@@ -304,11 +371,40 @@ __device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t parity, const
   return wait_or_abort(bar, parity, sm, status);
 }
 
-template <int JOB>
+template <int JOB, int P>
 __device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t dP, const ResidentStep *st, bool f16) {
   tc_fence_after();
   const uint64_t tk = sw128_desc(0, 16, 1024);
   const uint32_t dX = dP + 128u;
+  if (P == 2) {
+    // Two 64 x 64 tiles stacked along M (rows 64 j .. 64 j + 63 of a 128 x 64
+    // operand; X_s / S_s hold it K-major, one 128-byte swizzled block):
+    //   Gram / square  D_P (128 x 128) += Xs Xs^T, K = 64: the diagonal 64 x 64
+    //                  blocks are the two tiles' products, the rest is unused;
+    //   update         D_X (128 x 64) = Bop Xs, K = 128, Bop block-diagonal
+    //                  (zeros outside the tiles' blocks), Xs read MN-major.
+    // Every A operand is packed at TMEM columns dP + 192 .. dP + 255.
+    const uint32_t dA = dP + 192u;
+    if (JOB == kJobGram) {
+      const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
+      const uint32_t id = f16 ? idesc_f16(128, 128, 0, 0, 0, 0) : idesc_f16(128, 128, 1, 0, 0, 0);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) mma_ts(dP, dA + 8 * kk, desc_k(tk, x4, kk), id, kk > 0);
+    } else if (JOB == kJobSquare) {
+      const uint32_t s4 = smem_u32(sm.s(g)) >> 4;
+      const uint32_t id = idesc_f16(128, 128, f16 ? 0 : 1, 0, 0, st->neg2);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) mma_ts(dP, dA + 8 * kk, desc_k(tk, s4, kk), id, st->acc2 | (kk > 0));
+    } else {
+      const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
+      const uint64_t tmn = sw128_desc(0, kHalf, 1024);
+      const uint32_t id = f16 ? idesc_f16(128, 64, 0, 0, 1, 0) : idesc_f16(128, 64, 1, 0, 1, 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) mma_ts(dX, dA + 8 * kk, desc_mn(tmn, x4, kk), id, kk > 0);
+    }
+    mma_commit(sm.bar_mma(g));
+    return;
+  }
   // packed A operand: K columns 0..63 at region + [0, 32), 64..127 at region + [64, 96)
   if (JOB == kJobGram) {
     const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
@@ -354,6 +450,7 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
   const uint32_t dP = tmem + 256u * g;                 // D_P (lane 0); D_X = dP + 128
   const uint32_t tP = dP + ((q * 32) << 16);           // this warp's lanes of D_P
   const uint32_t tX = tP + 128u;                       // ... and of D_X
+  const uint32_t tA = tP + 192u;                       // ... and (P = 2) of the packed A operand
   uint8_t *Xs = sm.x(g), *Ss = sm.s(g), *Ws = sm.w(g);
   const bool step_mode = a.mode == 1;
   const bool has_w = step_mode && a.has_w;
@@ -395,6 +492,32 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     // M' (bf16, for the write-back) replaces G in S_s, so X_s is free for X_0 at once.
     // Columns outside this row's diagonal block are zero.
     float sumsq = 0.f;
+    if constexpr (P == 2) {   // stacked: this row's 64 columns, 32 per warp, fp32 at D_X columns 32 hf..
+      float v[32];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float m[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m[e] = 0.f;
+        if (row_valid) {
+          const uint32_t off = stage_off<P>(jr, rr, 4 * hf + k);
+          unpack8(*reinterpret_cast<const uint4 *>(Xs + off), m);
+          if (step_mode) {
+            float gg[8];
+            unpack8(*reinterpret_cast<const uint4 *>(Ss + off), gg);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m[e] = fmaf(a.mu, m[e], gg[e]);
+            *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(m);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[8 * k + e] = m[e];
+          sumsq = fmaf(m[e], m[e], sumsq);
+        }
+      }
+      tmem_st32(tX + 32 * hf, v);
+    } else
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       float v[32];
@@ -465,8 +588,13 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     if (gt == 0) *sm.fmt16(g) = f16 ? 1 : 0;   // read by the issuer after this group's next arrival
 
     // ---- operand g_0 X_0 = r(g_0 M' / rho) to X_s and (packed) to D_X
-    if (f16) tmem_row_to_op<0, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
-    else tmem_row_to_op<1, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
+    if constexpr (P == 2) {
+      if (f16) stack_tmem_to_op<0, true>(tX + 32 * hf, tA, Xs, r, hf, a.gamma0 / rho);
+      else stack_tmem_to_op<1, true>(tX + 32 * hf, tA, Xs, r, hf, a.gamma0 / rho);
+    } else {
+      if (f16) tmem_row_to_op<0, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
+      else tmem_row_to_op<1, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
+    }
     // M' must have left S_s before the first conversion (after MMA1) overwrites it
     if (step_mode && gt == 0) bulk_wait_read0();
     fence_proxy_async_smem();
@@ -492,7 +620,11 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
       if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
-      if (f16) {
+      if constexpr (P == 2) {   // the row's own tile block of D_P: columns 64 jr + 32 hf ..
+        const uint32_t src = tP + 64 * jr + 32 * hf;
+        if (f16) stack_tmem_to_op<0, true>(src, tA, Ss, r, hf, stp->s);
+        else stack_tmem_to_op<1, true>(src, tA, Ss, r, hf, stp->s);
+      } else if (f16) {
         if (stp->s == 1.f) tmem_row_to_op<0, false>(tP, tX, Ss, r, hf, 1.f);
         else tmem_row_to_op<0, true>(tP, tX, Ss, r, hf, stp->s);
       } else {
@@ -506,8 +638,13 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       bad = !wait_or_abort(sm.bar_mma(g), job++ & 1u, sm, a.status);
       if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
-      if (f16) tmem_row_to_tmem_op<0>(tP, r, hf, stp->beta, stp->a);
-      else tmem_row_to_tmem_op<1>(tP, r, hf, stp->beta, stp->a);
+      if constexpr (P == 2) {
+        if (f16) stack_row_to_bop<0>(tP, tA, r, hf, stp->beta, stp->a);
+        else stack_row_to_bop<1>(tP, tA, r, hf, stp->beta, stp->a);
+      } else {
+        if (f16) tmem_row_to_tmem_op<0>(tP, r, hf, stp->beta, stp->a);
+        else tmem_row_to_tmem_op<1>(tP, r, hf, stp->beta, stp->a);
+      }
       tc_fence_before();
       group_ready(sm, g, lane);
       // after MMA3: next operand r(xr D_X) = g_{t+1} X_{t+1} (xr = 1 for constant coefficients)
@@ -515,7 +652,10 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       if ((stop = __any_sync(0xffffffffu, bad))) break;
       tc_fence_after();
       if (t + 1 < a.K) {
-        if (f16) {
+        if constexpr (P == 2) {
+          if (f16) stack_tmem_to_op<0, true>(tX + 32 * hf, tA, Xs, r, hf, stp->xr);
+          else stack_tmem_to_op<1, true>(tX + 32 * hf, tA, Xs, r, hf, stp->xr);
+        } else if (f16) {
           if (stp->xr == 1.f) tmem_row_to_op<0, false>(tX, tX, Xs, r, hf, 1.f);
           else tmem_row_to_op<0, true>(tX, tX, Xs, r, hf, stp->xr);
         } else {
@@ -545,16 +685,17 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       if (__any_sync(0xffffffffu, bad)) break;
     }
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t c32 = 2 * hf + i;                  // 32-column group of the super-tile row
-      if (P == 1 || ((32 * c32) / T == jr && row_valid)) {
+    for (int i = 0; i < (P == 2 ? 1 : 2); ++i) {
+      // 32-column group of the super-tile row (P = 2: of the stacked row, at D_X columns 32 hf..)
+      const uint32_t c32 = P == 2 ? hf : 2 * hf + i;
+      if (P == 1 || (P == 2 && row_valid) || ((32 * c32) / T == jr && row_valid)) {
         float v[32];
         tmem_ld32(tX + 32 * c32, v);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint32_t cg = 4 * c32 + k;
-          const uint32_t off = stage_off<P>(jr, rr, cg - jr * (T / 8));
+          const uint32_t off = P == 2 ? stage_off<P>(jr, rr, cg) : stage_off<P>(jr, rr, cg - jr * (T / 8));
           const float *o = v + 8 * k;   // gamma_{K-1} O
           if (a.has_o) {
             float ov[8];
@@ -641,9 +782,9 @@ __device__ void issuer_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem
       const bool f16 = *sm.fmt16(g) != 0;
       const uint32_t dP = tmem + 256u * g;
       const ResidentStep *stp = &a.step[t];
-      if (jb == kJobGram) group_issue_mmas<kJobGram>(sm, g, dP, nullptr, f16);
-      else if (jb == kJobSquare) group_issue_mmas<kJobSquare>(sm, g, dP, stp, f16);
-      else group_issue_mmas<kJobUpdate>(sm, g, dP, stp, f16);
+      if (jb == kJobGram) group_issue_mmas<kJobGram, P>(sm, g, dP, nullptr, f16);
+      else if (jb == kJobSquare) group_issue_mmas<kJobSquare, P>(sm, g, dP, stp, f16);
+      else group_issue_mmas<kJobUpdate, P>(sm, g, dP, stp, f16);
       ++issued;
       // next job of this group: the Gram job of step t + 1, or of the next super-tile
       if (++jb == 3) {
