@@ -249,6 +249,57 @@ __device__ __forceinline__ void stack_row_to_bop(uint32_t tp, uint32_t pa, uint3
   tmem_wait_st();
 }
 
+// ---- stacked super-tiles of four 32 x 32 tiles (P = 4)
+// Rows 32 j .. 32 j + 31 of a 128 x 32 operand, K-major with 64-byte rows and
+// the 64-byte swizzle (again the TMA staging layout); the warp of half hf of a
+// row covers its columns 16 hf .. 16 hf + 15.
+__device__ __forceinline__ uint32_t sw64_off(uint32_t r, uint32_t c) { return r * 64u + ((c ^ ((r >> 1) & 3u)) << 4); }
+template <int F>
+__device__ __forceinline__ void stack4_tmem_to_op(uint32_t src, uint32_t pa, uint8_t *dst, uint32_t r, uint32_t hf,
+                                                  float scale) {
+  float v[16];
+  tmem_ld16(src, v);
+  tmem_wait_ld();
+  uint32_t p[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) p[e] = pack2_op<F>(v[2 * e] * scale, v[2 * e + 1] * scale);
+  tmem_st8(pa + 8u * hf, p);
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    *reinterpret_cast<uint4 *>(dst + sw64_off(r, 2u * hf + j)) = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+  tmem_wait_st();
+}
+// The block-diagonal A operand of the update for P = 4: row r's tile
+// j = r / 32 has its K values packed at columns 16 j .. 16 j + 15; the warp of
+// half hf writes packed columns pa + 32 hf .. + 31 (tiles 2 hf and 2 hf + 1).
+template <int F>
+__device__ __forceinline__ void stack4_row_to_bop(uint32_t tp, uint32_t pa, uint32_t r, uint32_t hf, float beta,
+                                                  float diag) {
+  const uint32_t jr = r >> 5;            // the same in the whole warp
+  uint32_t z[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) z[e] = 0u;
+  if ((jr >> 1) == hf) {
+    const uint32_t lane = r & 31u;       // the diagonal element's column in the tile
+    float v[32];
+    tmem_ld32(tp + 32u * jr, v);
+    tmem_wait_ld();
+    uint32_t p[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float a0 = fmaf(beta, v[2 * e], lane == 2u * e ? diag : 0.f);
+      const float a1 = fmaf(beta, v[2 * e + 1], lane == 2u * e + 1u ? diag : 0.f);
+      p[e] = pack2_op<F>(a0, a1);
+    }
+    tmem_st16(pa + 32u * hf + 16u * (jr & 1u), p);
+    tmem_st16(pa + 32u * hf + 16u * (1u - (jr & 1u)), z);
+  } else {
+    tmem_st16(pa + 32u * hf, z);
+    tmem_st16(pa + 32u * hf + 16u, z);
+  }
+  tmem_wait_st();
+}
+
 __device__ __forceinline__ bool use_smem_blocks(const ResidentArgs &a) {
   return a.smem_blocks != 0 && a.n_blocks <= kMaxSmemBlocks;
 }
@@ -405,6 +456,34 @@ __device__ __forceinline__ void group_issue_mmas(const Smem &sm, int g, uint32_t
     mma_commit(sm.bar_mma(g));
     return;
   }
+  if (P == 4) {
+    // Four 32 x 32 tiles stacked along M (rows 32 j .. 32 j + 31 of a 128 x 32
+    // operand, K-major with 64-byte rows and the 64-byte swizzle): Gram and
+    // square products with K = 32, the update with K = 128 (Bop
+    // block-diagonal) and N = 32, Xs read MN-major.
+    const uint32_t dA = dP + 192u;
+    const uint64_t tk64 = sw64_desc(0, 16, 512);
+    if (JOB == kJobGram) {
+      const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
+      const uint32_t id = f16 ? idesc_f16(128, 128, 0, 0, 0, 0) : idesc_f16(128, 128, 1, 0, 0, 0);
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) mma_ts(dP, dA + 8 * kk, tk64 + x4 + 2 * kk, id, kk > 0);
+    } else if (JOB == kJobSquare) {
+      const uint32_t s4 = smem_u32(sm.s(g)) >> 4;
+      const uint32_t id = idesc_f16(128, 128, f16 ? 0 : 1, 0, 0, st->neg2);
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) mma_ts(dP, dA + 8 * kk, tk64 + s4 + 2 * kk, id, st->acc2 | (kk > 0));
+    } else {
+      // K rows 16 kk .. 16 kk + 15: 1024 bytes on; one 32-column atom in N
+      const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
+      const uint64_t tmn64 = sw64_desc(0, 8192, 512);
+      const uint32_t id = f16 ? idesc_f16(128, 32, 0, 0, 1, 0) : idesc_f16(128, 32, 1, 0, 1, 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) mma_ts(dX, dA + 8 * kk, tmn64 + x4 + 64 * kk, id, kk > 0);
+    }
+    mma_commit(sm.bar_mma(g));
+    return;
+  }
   // packed A operand: K columns 0..63 at region + [0, 32), 64..127 at region + [64, 96)
   if (JOB == kJobGram) {
     const uint32_t x4 = smem_u32(sm.x(g)) >> 4;
@@ -517,6 +596,31 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
         }
       }
       tmem_st32(tX + 32 * hf, v);
+    } else if constexpr (P == 4) {   // stacked: this row's 32 columns, 16 per warp, fp32 at D_X columns 16 hf..
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        float m[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m[e] = 0.f;
+        if (row_valid) {
+          const uint32_t off = stage_off<P>(jr, rr, 2 * hf + k);
+          unpack8(*reinterpret_cast<const uint4 *>(Xs + off), m);
+          if (step_mode) {
+            float gg[8];
+            unpack8(*reinterpret_cast<const uint4 *>(Ss + off), gg);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m[e] = fmaf(a.mu, m[e], gg[e]);
+            *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(m);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[8 * k + e] = m[e];
+          sumsq = fmaf(m[e], m[e], sumsq);
+        }
+      }
+      tmem_st16(tX + 16 * hf, *reinterpret_cast<const uint32_t(*)[16]>(v));
     } else
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -591,6 +695,9 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
     if constexpr (P == 2) {
       if (f16) stack_tmem_to_op<0, true>(tX + 32 * hf, tA, Xs, r, hf, a.gamma0 / rho);
       else stack_tmem_to_op<1, true>(tX + 32 * hf, tA, Xs, r, hf, a.gamma0 / rho);
+    } else if constexpr (P == 4) {
+      if (f16) stack4_tmem_to_op<0>(tX + 16 * hf, tA, Xs, r, hf, a.gamma0 / rho);
+      else stack4_tmem_to_op<1>(tX + 16 * hf, tA, Xs, r, hf, a.gamma0 / rho);
     } else {
       if (f16) tmem_row_to_op<0, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
       else tmem_row_to_op<1, true>(tX, tX, Xs, r, hf, a.gamma0 / rho);
@@ -624,6 +731,10 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
         const uint32_t src = tP + 64 * jr + 32 * hf;
         if (f16) stack_tmem_to_op<0, true>(src, tA, Ss, r, hf, stp->s);
         else stack_tmem_to_op<1, true>(src, tA, Ss, r, hf, stp->s);
+      } else if constexpr (P == 4) {   // the row's own tile block of D_P: columns 32 jr + 16 hf ..
+        const uint32_t src = tP + 32 * jr + 16 * hf;
+        if (f16) stack4_tmem_to_op<0>(src, tA, Ss, r, hf, stp->s);
+        else stack4_tmem_to_op<1>(src, tA, Ss, r, hf, stp->s);
       } else if (f16) {
         if (stp->s == 1.f) tmem_row_to_op<0, false>(tP, tX, Ss, r, hf, 1.f);
         else tmem_row_to_op<0, true>(tP, tX, Ss, r, hf, stp->s);
@@ -641,6 +752,9 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       if constexpr (P == 2) {
         if (f16) stack_row_to_bop<0>(tP, tA, r, hf, stp->beta, stp->a);
         else stack_row_to_bop<1>(tP, tA, r, hf, stp->beta, stp->a);
+      } else if constexpr (P == 4) {
+        if (f16) stack4_row_to_bop<0>(tP, tA, r, hf, stp->beta, stp->a);
+        else stack4_row_to_bop<1>(tP, tA, r, hf, stp->beta, stp->a);
       } else {
         if (f16) tmem_row_to_tmem_op<0>(tP, r, hf, stp->beta, stp->a);
         else tmem_row_to_tmem_op<1>(tP, r, hf, stp->beta, stp->a);
@@ -655,6 +769,9 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
         if constexpr (P == 2) {
           if (f16) stack_tmem_to_op<0, true>(tX + 32 * hf, tA, Xs, r, hf, stp->xr);
           else stack_tmem_to_op<1, true>(tX + 32 * hf, tA, Xs, r, hf, stp->xr);
+        } else if constexpr (P == 4) {
+          if (f16) stack4_tmem_to_op<0>(tX + 16 * hf, tA, Xs, r, hf, stp->xr);
+          else stack4_tmem_to_op<1>(tX + 16 * hf, tA, Xs, r, hf, stp->xr);
         } else if (f16) {
           if (stp->xr == 1.f) tmem_row_to_op<0, false>(tX, tX, Xs, r, hf, 1.f);
           else tmem_row_to_op<0, true>(tX, tX, Xs, r, hf, stp->xr);
@@ -684,33 +801,42 @@ __device__ void group_main(const ResidentArgs &a, const Smem &sm, uint32_t tmem,
       if (gt == 0 && !bad) ++w_seen;
       if (__any_sync(0xffffffffu, bad)) break;
     }
+    // 8 values of gamma_{K-1} O for the staged tile at byte offset `off`: O and / or W'
+    auto emit8 = [&](uint32_t off, const float *o) {
+      if (a.has_o) {
+        float ov[8];
 #pragma unroll
-    for (int i = 0; i < (P == 2 ? 1 : 2); ++i) {
-      // 32-column group of the super-tile row (P = 2: of the stacked row, at D_X columns 32 hf..)
-      const uint32_t c32 = P == 2 ? hf : 2 * hf + i;
-      if (P == 1 || (P == 2 && row_valid) || ((32 * c32) / T == jr && row_valid)) {
-        float v[32];
-        tmem_ld32(tX + 32 * c32, v);
+        for (int e = 0; e < 8; ++e) ov[e] = a.oscale * o[e];
+        *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(ov);
+      }
+      if (has_w) {
+        const float lro = -a.lr * a.oscale;
+        float w[8];
+        unpack8(*reinterpret_cast<const uint4 *>(Ws + off), w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = fmaf(lro, o[e], w[e]);
+        *reinterpret_cast<uint4 *>(Ws + off) = pack8_bf16(w);
+      }
+    };
+    if constexpr (P == 4) {   // stacked: this row's 32 columns, 16 per warp, at D_X columns 16 hf..
+      if (row_valid) {
+        float v[16];
+        tmem_ld16(tX + 16 * hf, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t cg = 4 * c32 + k;
-          const uint32_t off = P == 2 ? stage_off<P>(jr, rr, cg) : stage_off<P>(jr, rr, cg - jr * (T / 8));
-          const float *o = v + 8 * k;   // gamma_{K-1} O
-          if (a.has_o) {
-            float ov[8];
+        for (int k = 0; k < 2; ++k) emit8(stage_off<P>(jr, rr, 2 * hf + k), v + 8 * k);
+      }
+    } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ov[e] = a.oscale * o[e];
-            *reinterpret_cast<uint4 *>(Ss + off) = pack8_bf16(ov);
-          }
-          if (has_w) {
-            const float lro = -a.lr * a.oscale;
-            float w[8];
-            unpack8(*reinterpret_cast<const uint4 *>(Ws + off), w);
+      for (int i = 0; i < (P == 2 ? 1 : 2); ++i) {
+        // 32-column group of the super-tile row (P = 2: of the stacked row, at D_X columns 32 hf..)
+        const uint32_t c32 = P == 2 ? hf : 2 * hf + i;
+        if (P == 1 || row_valid) {
+          float v[32];
+          tmem_ld32(tX + 32 * c32, v);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = fmaf(lro, o[e], w[e]);
-            *reinterpret_cast<uint4 *>(Ws + off) = pack8_bf16(w);
-          }
+          for (int k = 0; k < 4; ++k) emit8(stage_off<P>(jr, rr, 4 * c32 + k), v + 8 * k);
         }
       }
     }

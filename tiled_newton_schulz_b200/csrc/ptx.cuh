@@ -208,6 +208,21 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 // 32 lanes x 16 consecutive 32-bit columns from 16 registers per thread.
+// 32 lanes x 16 consecutive 32-bit columns -> 16 registers per thread
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t *r = reinterpret_cast<uint32_t *>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -333,6 +348,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo,
   d |= (uint64_t)1 << 46;   // version
   d |= (uint64_t)2 << 61;   // SWIZZLE_128B
   return d;
+}
+// The same with the 64-byte swizzle (layout type 4): rows of 64 bytes, the
+// pattern repeating every 8 rows (512 bytes).
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  return (sw128_desc(smem_addr, lbo, sbo) & ~((uint64_t)7 << 61)) | ((uint64_t)4 << 61);
 }
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 //   ab_fmt: 0 = fp16, 1 = bf16;  a_mn / b_mn: operand is MN-major;  neg_a: negate A.
