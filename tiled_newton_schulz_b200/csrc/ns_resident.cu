@@ -6,11 +6,14 @@
 // Tiles up to 128 x 128 are zero-padded to 128 x 128 (exactly the same map: a
 // zero border stays zero through X X^T, A^2 and B X and leaves ||X||_F alone;
 // and the transpose of a tall tile is not needed because NS(X^T) = NS(X)^T).
-// For T = 64 and T = 32, P = 128 / T consecutive tiles share one 128 x 128
-// "super-tile" as diagonal blocks, each normalised by its own norm: X X^T,
-// A^2 and B X of a block-diagonal matrix are block-diagonal with exactly the
-// blocks' own products (the off-diagonal zeros stay exact zeros in fp32), so
-// each block goes through exactly its own map.
+// For T = 64 and T = 32, P = 128 / T consecutive tiles share one "super-tile",
+// stacked along M as rows T j .. T j + T - 1 of a 128 x T operand, each
+// normalised by its own norm.  The Gram and square products then run with
+// K = T (D_P = Xs Xs^T, 128 x 128: its diagonal T x T blocks are the tiles'
+// own products, the rest is never read), and the update D_X = Bop Xs with
+// K = 128 and N = T, where the packed A operand Bop is block-diagonal (zeros
+// outside each row's tile), so each tile goes through exactly its own map
+// with 2x (T = 64) or 4x (T = 32) the MMA work of its own products.
 //
 // One persistent CTA per SM runs two independent tile "groups" of 8 warps
 // (two per TMEM lane quarter, each owning 64 of a row's 128 columns), so that
