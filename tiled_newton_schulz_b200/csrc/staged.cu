@@ -328,8 +328,8 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
 }
 
 // ---------------------------------------------------------------- tcgen05 GEMM
-// A CTA computes a 128 x BN output tile (BN = 128, or 256 for products that
-// are not symmetric and have N a multiple of 256: a 128 x 256 x 16 MMA reads
+// A CTA computes a 128 x BN output tile (BN = 256 when N is a multiple of
+// 256, and at least 2048 for a symmetric product; else 128: a 128 x 256 x 16 MMA reads
 // 12 KB of operands from shared memory in 128 cycles where two 128 x 128 x 16
 // ones read 16 KB, which keeps the operand traffic under the shared-memory
 // bandwidth).  Pipeline depth for 128-column tiles: 3 stages for long K; 2
@@ -363,13 +363,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t n0 = blockIdx.x * BN, m0 = blockIdx.y * 128;
   const int32_t z = blockIdx.z;
-  if (a.ep.sym) {   // blockIdx.x enumerates the tiles (ti, tj), tj <= ti, row by row
+  if (a.ep.sym && BN == 128) {   // blockIdx.x enumerates the tiles (ti, tj), tj <= ti, row by row
     const int32_t k = blockIdx.x;
     int32_t ti = static_cast<int32_t>((sqrtf(8.f * k + 1.f) - 1.f) * 0.5f);
     while ((ti + 1) * (ti + 2) / 2 <= k) ++ti;
     while (ti * (ti + 1) / 2 > k) --ti;
     m0 = ti * 128;
     n0 = (k - ti * (ti + 1) / 2) * 128;
+  } else if (a.ep.sym) {
+    // 128 x 256 tiles reaching the lower triangle: row tile ti holds
+    // ti / 2 + 1 of them (columns 0 .. 256 (ti / 2) + 255), row by row
+    const int32_t k = blockIdx.x;
+    int32_t ti = 0, base = 0;
+    while (base + ti / 2 + 1 <= k) {
+      base += ti / 2 + 1;
+      ++ti;
+    }
+    m0 = ti * 128;
+    n0 = (k - base) * 256;
   } else if (gridDim.y > 1) {
     // Grouped order: the CTAs launched together cover bands of up to 32 row
     // tiles, row tile fastest, so one wave shares each B column panel among
@@ -383,7 +394,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     m0 = static_cast<int32_t>((g * G + r % gm) * 128);
     n0 = static_cast<int32_t>((r / gm) * BN);
   }
-  const bool mirror = a.ep.sym && m0 != n0;
+  // symmetric products: each 128-column block of the tile below the diagonal
+  // is also written mirrored, the diagonal block as it is, and a block above
+  // the diagonal (in a 256-column tile on the diagonal) not at all: its
+  // mirror image comes from the tile below
+  const int32_t ti = m0 / 128;
   const int nk = static_cast<int>(a.K / 64);
 
   if (threadIdx.x == 0) {
@@ -444,6 +459,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int64_t obase = z * a.ep.stride + static_cast<int64_t>(m0 + row) * a.ep.N + n0;
 #pragma unroll 1
       for (int i = 0; i < BN / 32; ++i) {
+        const int32_t ct = (n0 + 32 * i) / 128;   // 128-column block of the output
+        if (a.ep.sym && ct > ti) break;          // above the diagonal (the tile's last block)
+        const bool mirror = a.ep.sym && ct < ti;
         float v[32];
         tmem_ld32(taddr + 32 * i, v);
         tmem_wait_ld();
@@ -581,7 +599,10 @@ cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int6
   a.K = K;
   a.ep = to_epi(ep, M, N);
   a.status = status;
-  const int BN = (!a.ep.sym && N % 256 == 0) ? 256 : 128;
+  // 256-column tiles when N allows; for a symmetric product only from N = 2048,
+  // where the tiles on the diagonal, half above it, cost at most 6% extra
+  // work (at N = 1024 the extra 11% outweighed the faster MMAs: measured)
+  const int BN = (N % 256 == 0 && (!a.ep.sym || N >= 2048)) ? 256 : 128;
   CUtensorMap ma, mb;
   if (!make_batch_map(&ma, A, batch, 64, 128)) return cudaErrorInvalidValue;
   if (b_trans) {
@@ -591,9 +612,11 @@ cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int6
   }
   a.idesc = idesc_f16(128, static_cast<uint32_t>(BN), A.dtype == HIMUON_FP16 ? 0u : 1u, 0, b_trans ? 0u : 1u, 0);
   dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(M / 128), static_cast<unsigned>(batch));
-  if (a.ep.sym) {
+  if (a.ep.sym) {   // the tiles reaching the lower triangle (see the kernel)
     const int64_t nt = M / 128;
-    grid = dim3(static_cast<unsigned>(nt * (nt + 1) / 2), 1, static_cast<unsigned>(batch));
+    int64_t count = 0;
+    for (int64_t ti = 0; ti < nt; ++ti) count += BN == 128 ? ti + 1 : ti / 2 + 1;
+    grid = dim3(static_cast<unsigned>(count), 1, static_cast<unsigned>(batch));
   }
   cudaError_t e;
   auto go = [&](auto kern, uint32_t smem) -> cudaError_t {
