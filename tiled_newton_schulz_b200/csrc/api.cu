@@ -534,14 +534,20 @@ size_t chunk_limit(size_t ws_bytes, const himuon_ns_params &p) {
   return lim;
 }
 
-// Tiles per chunk of a class under the limit (0 if even one tile does not fit).
+// Tiles per chunk of a class under the limit (0 if even one tile does not fit):
+// the fewest chunks the limit allows, of equal size (a last chunk of a tile or
+// two would run every product of the call once more at a tiny batch).
 int64_t chunk_tiles(const TileClass &c, size_t limit, int compute, bool gram) {
-  const size_t one = ws_layout(c.n, c.m, 1, compute, gram).total;
-  int64_t k = static_cast<int64_t>(limit / one);
-  k = std::min<int64_t>(k, static_cast<int64_t>(c.tiles.size()));
-  k = std::min<int64_t>(k, 65535);
-  while (k > 0 && ws_layout(c.n, c.m, k, compute, gram).total > limit) --k;
-  return k;
+  const int64_t tiles = static_cast<int64_t>(c.tiles.size());
+  if (tiles < 1 || ws_layout(c.n, c.m, 1, compute, gram).total > limit) return 0;
+  int64_t lo = 1, hi = std::min<int64_t>(tiles, 65535);   // the workspace grows with the tile count
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) / 2;
+    if (ws_layout(c.n, c.m, mid, compute, gram).total <= limit) lo = mid;
+    else hi = mid - 1;
+  }
+  const int64_t chunks = (tiles + lo - 1) / lo;
+  return (tiles + chunks - 1) / chunks;
 }
 
 int64_t staged_ws_bytes(const Plan &plan, int op, int compute) {
