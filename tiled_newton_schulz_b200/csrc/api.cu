@@ -587,6 +587,7 @@ Epilogue epi(float alpha, float beta, const float *c32, float *out32, void *out1
   e.alpha = alpha;
   e.beta = beta;
   e.c32 = c32;
+  e.c16 = nullptr;
   e.out32 = out32;
   e.out16 = out16;
   e.out16_dtype = dt;
@@ -660,12 +661,16 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
         for (int t = 0; t < p.steps && rc == HIMUON_OK; ++t) {
           const float a = p.coeffs[3 * t], b = p.coeffs[3 * t + 1], cc = p.coeffs[3 * t + 2];
           // A = X X^T
-          rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, sym(epi(1.f, 0.f, nullptr, a32, a16, dt16)));
+          rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc,
+                      sym(epi(1.f, 0.f, nullptr, f32 ? a32 : nullptr, a16, dt16)));
           if (rc) break;
-          // 16-bit operands: Bop = r(b A + c A A + a I), and X <- r(Bop X) (fp32
-          // accumulation, the whole update in one product, as on chip).
+          // 16-bit operands: Bop = r(b r(A) + c r(A) r(A) + a I), and X <- r(Bop X)
+          // (fp32 accumulation, the whole update in one product, as on chip; the
+          // b A term reads the same 16-bit A as the product's operands, whose
+          // rounding is of the size of Bop's own).
           // fp32: B' = b A + c A A + (a - 1) I, and X <- X + B' X on the fp32 master.
-          Epilogue e2 = epi(cc, b, a32, f32 ? static_cast<float *>(bop) : nullptr, f32 ? nullptr : bop, dt16);
+          Epilogue e2 = epi(cc, b, f32 ? a32 : nullptr, f32 ? static_cast<float *>(bop) : nullptr, f32 ? nullptr : bop, dt16);
+          if (!f32) e2.c16 = a16;
           e2.diag = f32 ? a - 1.f : a;
           e2.sym = 1;
           rc = ops.mm(f32 ? static_cast<void *>(a32) : a16, n, n, f32 ? static_cast<void *>(a32) : a16, n, n, 0, n, n,

@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(256) unpack_kernel(const UnpackArgs a, int32_t
 struct EpiArgs {
   float alpha, beta, diag;
   const float *c32;
+  const void *c16;   // 16-bit C term (out16_dtype), tensor-core path only
   float *out32;
   void *out16;
   int32_t out16_dtype;
@@ -306,6 +307,28 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
     const float4 c0 = *reinterpret_cast<const float4 *>(e.c32 + o);
     const float4 c1 = *reinterpret_cast<const float4 *>(e.c32 + o + 4);
     const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = fmaf(e.alpha, acc[i], e.beta * cc[i]);
+  } else if (e.c16) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(e.c16) + o);
+    float cc[8];
+    if (e.out16_dtype == HIMUON_FP16) {
+      const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        cc[2 * i] = f.x;
+        cc[2 * i + 1] = f.y;
+      }
+    } else {
+      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        cc[2 * i] = f.x;
+        cc[2 * i + 1] = f.y;
+      }
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = fmaf(e.alpha, acc[i], e.beta * cc[i]);
   } else {
@@ -578,6 +601,7 @@ EpiArgs to_epi(const Epilogue &e, int64_t M, int64_t N) {
   a.beta = e.beta;
   a.diag = e.diag;
   a.c32 = e.c32;
+  a.c16 = e.c16;
   a.out32 = e.out32;
   a.out16 = e.out16;
   a.out16_dtype = e.out16_dtype;

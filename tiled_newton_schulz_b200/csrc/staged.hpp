@@ -24,6 +24,7 @@ struct Epilogue {
   float alpha, beta;
   float diag;       // added on the diagonal of each (square) output matrix
   const float *c32;
+  const void *c16;      // the C term in 16 bits (out16_dtype) instead of c32 (nullptr: none)
   float *out32;
   void *out16;
   int32_t out16_dtype;
