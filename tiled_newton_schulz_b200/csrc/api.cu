@@ -505,7 +505,7 @@ WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, bool gram) 
     L.x16a = take(2 * nm);
     L.x16b = take(2 * nm);
   }
-  L.a32 = take(4 * nn);
+  if (f32 || gram) L.a32 = take(4 * nn);   // (the 16-bit NS path keeps A in 16 bits only)
   if (!f32) L.a16 = take(2 * nn);
   if (!gram) {
     if (f32) L.b32 = take(4 * nn);
@@ -623,7 +623,7 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       const WsLayout L = ws_layout(n, m, bc, compute, gram);
       float *x32[2] = {reinterpret_cast<float *>(W + L.x32a), f32 ? reinterpret_cast<float *>(W + L.x32b) : nullptr};
       void *x16[2] = {f32 ? nullptr : W + L.x16a, f32 ? nullptr : W + L.x16b};
-      float *a32 = reinterpret_cast<float *>(W + L.a32);
+      float *a32 = (f32 || gram) ? reinterpret_cast<float *>(W + L.a32) : nullptr;
       void *a16 = f32 ? nullptr : W + L.a16;
       const DevTile *tiles = plan.d_tiles + c.dev_offset + t0;
       if (c.padded) HIMUON_TRY(cudaMemsetAsync(x32[0], 0, sizeof(float) * n * m * bc, stream));
