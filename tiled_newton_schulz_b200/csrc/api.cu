@@ -173,11 +173,11 @@ int check_call(const CallMats &cm, const himuon_split *splits) {
 enum PathKind { kPathResident = 0, kPathStaged = 1, kPathPair = 2 };
 
 struct TileClass {
-  int64_t n, m;          // padded iterate shape (n <= m)
-  bool padded;           // some tile of the class is smaller than n x m
-  bool thin;             // every tile of the class has a short side <= kThinSide
+  int64_t n = 0, m = 0;      // padded iterate shape (n <= m)
+  bool padded = false;       // some tile of the class is smaller than n x m
+  bool thin = false;         // every tile of the class has a short side <= kThinSide
   std::vector<DevTile> tiles;
-  int64_t dev_offset;    // index of the class's first DevTile in the device table
+  int64_t dev_offset = 0;    // index of the class's first DevTile in the device table
 };
 
 struct Plan {
