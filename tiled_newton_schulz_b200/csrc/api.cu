@@ -485,7 +485,7 @@ int check_device() {
 
 // ---------------------------------------------------------------- workspace layout
 struct WsLayout {
-  size_t x32a, x32b, x16a, x16b, a32, a16, b32, b16, q32, q16a, q16b, z32, z16, rz32, rz16, partial, total;
+  size_t x32a, x32b, x16a, x16b, a32, a16, b32, b16, q32, q16a, q16b, z32, z16, rz32, rz16, partial, scale, total;
 };
 
 WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, bool gram) {
@@ -524,6 +524,7 @@ WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, bool gram) 
   }
   const int64_t parts = (std::max(n, m) + 31) / 32;
   L.partial = take(4 * parts * count);
+  L.scale = take(8 * count);   // per-tile 1 / rho and 1 / rho^2 (the bf16 path)
   L.total = off;
   return L;
 }
@@ -588,6 +589,7 @@ Epilogue epi(float alpha, float beta, const float *c32, float *out32, void *out1
   e.beta = beta;
   e.c32 = c32;
   e.c16 = nullptr;
+  e.alpha_batch = nullptr;
   e.out32 = out32;
   e.out16 = out16;
   e.out16_dtype = dt;
@@ -626,14 +628,24 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       float *a32 = (f32 || gram) ? reinterpret_cast<float *>(W + L.a32) : nullptr;
       void *a16 = f32 ? nullptr : W + L.a16;
       const DevTile *tiles = plan.d_tiles + c.dev_offset + t0;
-      if (c.padded) HIMUON_TRY(cudaMemsetAsync(x32[0], 0, sizeof(float) * n * m * bc, stream));
+      // bf16 NS: the input goes to the bf16 operand as it is and the first
+      // step's two products over X apply 1 / rho^2 and 1 / rho in their
+      // epilogues (no normalisation pass, no fp32 copy of the input).  fp16
+      // keeps the pass: an unnormalised input may not fit fp16's range.
+      const bool prescale = !f32 && !gram && dt16 == HIMUON_BF16;
+      float *inv = reinterpret_cast<float *>(W + L.scale), *inv2 = inv + bc;
+      if (c.padded) {
+        if (prescale) HIMUON_TRY(cudaMemsetAsync(x16[0], 0, 2 * n * m * bc, stream));
+        else HIMUON_TRY(cudaMemsetAsync(x32[0], 0, sizeof(float) * n * m * bc, stream));
+      }
       PackArgs pk;
       pk.blocks = plan.d_blocks;
       pk.tiles = tiles;
       pk.n_tiles = bc;
       pk.n = n;
       pk.m = m;
-      pk.x32 = x32[0];
+      pk.x32 = prescale ? nullptr : x32[0];
+      pk.x16 = prescale ? x16[0] : nullptr;
       pk.partial = reinterpret_cast<float *>(W + L.partial);
       pk.parts = static_cast<int32_t>((std::max(n, m) + 31) / 32);
       pk.mode = step ? 1 : 0;
@@ -650,7 +662,8 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       na.keep32 = f32 ? 1 : 0;   // the 16-bit paths (NS and Gram NS) read only the 16-bit copy
       na.eps = p.eps;
       na.safety = safety;
-      HIMUON_TRY(launch_normalize(na, stream));
+      if (prescale) HIMUON_TRY(launch_tile_scales(pk.partial, pk.parts, bc, p.eps, safety, inv, inv2, stream));
+      else HIMUON_TRY(launch_normalize(na, stream));
       int cur = 0;  // which x buffer holds the current operand
       float *xfinal = x32[0];
       int rc = HIMUON_OK;
@@ -660,9 +673,10 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
         void *bop = f32 ? static_cast<void *>(W + L.b32) : W + L.b16;
         for (int t = 0; t < p.steps && rc == HIMUON_OK; ++t) {
           const float a = p.coeffs[3 * t], b = p.coeffs[3 * t + 1], cc = p.coeffs[3 * t + 2];
-          // A = X X^T
-          rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc,
-                      sym(epi(1.f, 0.f, nullptr, f32 ? a32 : nullptr, a16, dt16)));
+          // A = X X^T  (step 0 of the bf16 path: (X X^T) / rho^2)
+          Epilogue e1 = sym(epi(1.f, 0.f, nullptr, f32 ? a32 : nullptr, a16, dt16));
+          if (prescale && t == 0) e1.alpha_batch = inv2;
+          rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, e1);
           if (rc) break;
           // 16-bit operands: Bop = r(b r(A) + c r(A) r(A) + a I), and X <- r(Bop X)
           // (fp32 accumulation, the whole update in one product, as on chip; the
@@ -683,9 +697,11 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
             xfinal = x32[cur];
           } else {
             // the 16-bit operand for the next step, or the fp32 result after the last
+            // (step 0 of the bf16 path: Bop (X / rho) = (Bop X) / rho)
             const bool last = t + 1 == p.steps;
-            rc = ops.mm(bop, n, n, x16[cur], n, m, 0, n, m, n, bc,
-                        epi(1.f, 0.f, nullptr, last ? x32[0] : nullptr, last ? nullptr : x16[1 - cur], dt16));
+            Epilogue e3 = epi(1.f, 0.f, nullptr, last ? x32[0] : nullptr, last ? nullptr : x16[1 - cur], dt16);
+            if (prescale && t == 0) e3.alpha_batch = inv;
+            rc = ops.mm(bop, n, n, x16[cur], n, m, 0, n, m, n, bc, e3);
             cur = 1 - cur;
           }
         }

@@ -99,7 +99,8 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
   const int32_t rpp = (tl.h + a.parts - 1) / a.parts;
   const int32_t i0 = blockIdx.x * rpp;
   const int32_t i1 = min(tl.h, i0 + rpp);
-  float *x = a.x32 + t * a.n * a.m;
+  float *x = a.x32 ? a.x32 + t * a.n * a.m : nullptr;
+  __nv_bfloat16 *xh = a.x32 ? nullptr : static_cast<__nv_bfloat16 *>(a.x16) + t * a.n * a.m;
   float ss = 0.f;
   if (i0 < i1) {
     const void *src = b.ptr[kRoleIn];
@@ -126,7 +127,14 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
-      if (tl.transposed) {
+      if (xh) {
+        if (tl.transposed) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xh[static_cast<int64_t>(j + e) * a.m + i] = __float2bfloat16_rn(v[e]);
+        } else {
+          st8_16(xh, HIMUON_BF16, static_cast<int64_t>(i) * a.m + j, v);
+        }
+      } else if (tl.transposed) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[static_cast<int64_t>(j + e) * a.m + i] = v[e];
       } else {
@@ -144,7 +152,9 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
         st_elem(b.ptr[kRoleIn], dt, gi, v);
       }
       ss = fmaf(v, v, ss);
-      x[tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j] = v;
+      const int64_t o = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
+      if (xh) xh[o] = __float2bfloat16_rn(v);
+      else x[o] = v;
     }
   }
   const float s = block_sum<256>(ss, scratch);
@@ -250,6 +260,7 @@ struct EpiArgs {
   float alpha, beta, diag;
   const float *c32;
   const void *c16;   // 16-bit C term (out16_dtype), tensor-core path only
+  const float *alpha_batch;   // per-matrix alpha (tensor-core path only; nullptr: alpha)
   float *out32;
   void *out16;
   int32_t out16_dtype;
@@ -302,13 +313,14 @@ __device__ __forceinline__ void epi_put8(const EpiArgs &e, float *out32, void *o
 // hold consecutive rows, so each of these scalar stores is coalesced).
 __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t row, int64_t col, const float *acc,
                                            bool mirror = false, int64_t om = 0) {
+  const float alpha = e.alpha_batch ? e.alpha_batch[o / e.stride] : e.alpha;
   float v[8];
   if (e.c32) {
     const float4 c0 = *reinterpret_cast<const float4 *>(e.c32 + o);
     const float4 c1 = *reinterpret_cast<const float4 *>(e.c32 + o + 4);
     const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = fmaf(e.alpha, acc[i], e.beta * cc[i]);
+    for (int i = 0; i < 8; ++i) v[i] = fmaf(alpha, acc[i], e.beta * cc[i]);
   } else if (e.c16) {
     const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(e.c16) + o);
     float cc[8];
@@ -330,10 +342,10 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
       }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = fmaf(e.alpha, acc[i], e.beta * cc[i]);
+    for (int i = 0; i < 8; ++i) v[i] = fmaf(alpha, acc[i], e.beta * cc[i]);
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = e.alpha * acc[i];
+    for (int i = 0; i < 8; ++i) v[i] = alpha * acc[i];
   }
   const bool on_diag = row >= col && row < col + 8;
   if (e.diag != 0.f && on_diag) {
@@ -602,6 +614,7 @@ EpiArgs to_epi(const Epilogue &e, int64_t M, int64_t N) {
   a.diag = e.diag;
   a.c32 = e.c32;
   a.c16 = e.c16;
+  a.alpha_batch = e.alpha_batch;
   a.out32 = e.out32;
   a.out16 = e.out16;
   a.out16_dtype = e.out16_dtype;
@@ -681,6 +694,25 @@ cudaError_t launch_pack(const PackArgs &a, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(a.parts), static_cast<unsigned>(a.n_tiles));
   count_launch();
   pack_kernel<<<grid, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+__global__ void tile_scales_kernel(const float *partial, int32_t parts, int64_t n_tiles, float eps, float safety,
+                                   float *inv, float *inv2) {
+  const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (t >= n_tiles) return;
+  float s = 0.f;
+  for (int p = 0; p < parts; ++p) s += partial[t * parts + p];   // the order normalize_kernel sums in
+  const float v = 1.0f / ((sqrtf(s) + eps) * safety);
+  inv[t] = v;
+  inv2[t] = v * v;
+}
+
+cudaError_t launch_tile_scales(const float *partial, int32_t parts, int64_t n_tiles, float eps, float safety,
+                               float *inv, float *inv2, cudaStream_t stream) {
+  count_launch();
+  tile_scales_kernel<<<static_cast<unsigned>((n_tiles + 255) / 256), 256, 0, stream>>>(partial, parts, n_tiles, eps,
+                                                                                     safety, inv, inv2);
   return cudaGetLastError();
 }
 

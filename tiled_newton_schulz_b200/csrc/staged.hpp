@@ -25,6 +25,7 @@ struct Epilogue {
   float diag;       // added on the diagonal of each (square) output matrix
   const float *c32;
   const void *c16;      // the C term in 16 bits (out16_dtype) instead of c32 (nullptr: none)
+  const float *alpha_batch;   // per-matrix alpha (replaces alpha; tensor-core path only)
   float *out32;
   void *out16;
   int32_t out16_dtype;
@@ -54,7 +55,8 @@ struct PackArgs {
   const DevTile *tiles;   // tiles of this chunk
   int64_t n_tiles;
   int64_t n, m;           // padded iterate shape (n <= m), row-major n x m per tile
-  float *x32;             // n_tiles * n * m
+  float *x32;             // n_tiles * n * m (fp32 iterate), or nullptr when x16 takes the values
+  void *x16;              // bf16 copy instead of x32 (the bf16 path scales in its first products)
   float *partial;         // n_tiles * parts
   int32_t parts;          // partial sums per tile (row slices of the source tile)
   int32_t mode;           // 0: NS input; 1: momentum (M' = mu M + G written back to M)
@@ -74,6 +76,9 @@ struct NormArgs {
   float eps, safety;
 };
 cudaError_t launch_normalize(const NormArgs &a, cudaStream_t stream);
+// inv[t] = 1 / ((sqrt(sum of tile t's partial sums) + eps) * safety), inv2[t] = inv[t]^2
+cudaError_t launch_tile_scales(const float *partial, int32_t parts, int64_t n_tiles, float eps, float safety,
+                               float *inv, float *inv2, cudaStream_t stream);
 
 struct UnpackArgs {
   const DevBlock *blocks;
