@@ -363,77 +363,89 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
 }
 
 // ---------------------------------------------------------------- tcgen05 GEMM
-// A CTA computes a 128 x BN output tile (BN = 256 when N is a multiple of
-// 256, and at least 2048 for a symmetric product; else 128: a 128 x 256 x 16 MMA reads
-// 12 KB of operands from shared memory in 128 cycles where two 128 x 128 x 16
-// ones read 16 KB, which keeps the operand traffic under the shared-memory
-// bandwidth).  Pipeline depth for 128-column tiles: 3 stages for long K; 2
-// when K <= 256 (at most 4 k-blocks), which lets more CTAs share an SM and
-// hide each other's latency; 256-column tiles always take 2.
+// A persistent kernel, one CTA per SM, computes 128 x BN output tiles (BN =
+// 256 when N is a multiple of 256, and at least 2048 for a symmetric product;
+// else 128: a 128 x 256 x 16 MMA reads 12 KB of operands from shared memory in
+// 128 cycles where two 128 x 128 x 16 ones read 16 KB, which keeps the operand
+// traffic under the shared-memory bandwidth).  Warp 0 streams the operands of
+// its tiles, one after the other, through a ring of stages (TMA); warp 1
+// issues each tile's MMAs into one of two TMEM accumulators; warps 2..9 drain
+// the other accumulator (the previous tile) meanwhile, so the epilogue runs
+// under the next tile's main loop.  Two warps share each 32-lane quarter of
+// the accumulator, one per half of its columns: eight warps keep enough
+// stores in flight that the epilogue of a short-K tile still hides under the
+// next one's MMAs.
 constexpr uint32_t kStageA = 16384;
 template <int BN>
 __host__ __device__ constexpr uint32_t stage_bytes() { return kStageA + BN * 128u; }
-template <int STAGES, int BN>
-constexpr uint32_t gemm_smem() { return STAGES * stage_bytes<BN>() + 128 + 1024; }
-constexpr int kGemmThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+template <int BN>
+__host__ __device__ constexpr int gemm_stages() { return BN == 256 ? 4 : 6; }
+template <int BN>
+constexpr uint32_t gemm_smem() { return gemm_stages<BN>() * stage_bytes<BN>() + 256 + 1024; }
+constexpr int kGemmThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 
 struct GemmTcArgs {
   int64_t K;
   uint32_t idesc;
   EpiArgs ep;
   int *status;
+  int64_t tiles_per_matrix;   // output tiles of one matrix of the batch
+  int64_t n_tiles;            // tiles_per_matrix * batch
+  int32_t gx, gy;             // output tiles along N and M (non-symmetric products)
 };
 
-template <int B_MN, int kStages, int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                   const GemmTcArgs a) {
-  constexpr uint32_t kStageBytes = stage_bytes<BN>();
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + kStages * kStageBytes);
-  uint64_t *empty = full + kStages;
-  uint64_t *done = empty + kStages;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t n0 = blockIdx.x * BN, m0 = blockIdx.y * 128;
-  const int32_t z = blockIdx.z;
-  if (a.ep.sym && BN == 128) {   // blockIdx.x enumerates the tiles (ti, tj), tj <= ti, row by row
-    const int32_t k = blockIdx.x;
-    int32_t ti = static_cast<int32_t>((sqrtf(8.f * k + 1.f) - 1.f) * 0.5f);
+// Output tile `idx` of the launch: its matrix z and corner (m0, n0).
+template <int BN>
+__device__ __forceinline__ void gemm_tile(const GemmTcArgs &a, int64_t idx, int32_t &m0, int32_t &n0, int32_t &z) {
+  z = static_cast<int32_t>(idx / a.tiles_per_matrix);
+  const int64_t k = idx - static_cast<int64_t>(z) * a.tiles_per_matrix;
+  if (a.ep.sym && BN == 128) {   // the tiles (ti, tj), tj <= ti, row by row
+    int32_t ti = static_cast<int32_t>((sqrtf(8.f * static_cast<float>(k) + 1.f) - 1.f) * 0.5f);
     while ((ti + 1) * (ti + 2) / 2 <= k) ++ti;
     while (ti * (ti + 1) / 2 > k) --ti;
     m0 = ti * 128;
-    n0 = (k - ti * (ti + 1) / 2) * 128;
+    n0 = static_cast<int32_t>(k - ti * (ti + 1) / 2) * 128;
   } else if (a.ep.sym) {
     // 128 x 256 tiles reaching the lower triangle: row tile ti holds
     // ti / 2 + 1 of them (columns 0 .. 256 (ti / 2) + 255), row by row
-    const int32_t k = blockIdx.x;
-    int32_t ti = 0, base = 0;
+    int32_t ti = 0;
+    int64_t base = 0;
     while (base + ti / 2 + 1 <= k) {
       base += ti / 2 + 1;
       ++ti;
     }
     m0 = ti * 128;
-    n0 = (k - base) * 256;
-  } else if (gridDim.y > 1) {
-    // Grouped order: the CTAs launched together cover bands of up to 32 row
-    // tiles, row tile fastest, so one wave shares each B column panel among
-    // the band's rows and keeps the band's A row panels in L2 while B streams
-    // through once (row-major order re-read all of B for every ~2 row tiles).
-    const int64_t gx = gridDim.x, gy = gridDim.y;
-    const int64_t L = static_cast<int64_t>(blockIdx.y) * gx + blockIdx.x;   // launch order
+    n0 = static_cast<int32_t>(k - base) * 256;
+  } else {
+    // Grouped order: consecutive tiles cover bands of up to 32 row tiles, row
+    // tile fastest, so the tiles in flight together share each B column panel
+    // among the band's rows and keep the band's A row panels in L2 while B
+    // streams through once (row-major order re-read all of B for every ~2 row
+    // tiles).
+    const int64_t gx = a.gx, gy = a.gy;
     const int64_t G = gy < 32 ? gy : 32;
-    const int64_t per = G * gx, g = L / per, r = L % per;
+    const int64_t per = G * gx, g = k / per, r = k % per;
     const int64_t gm = (gy - g * G) < G ? (gy - g * G) : G;
     m0 = static_cast<int32_t>((g * G + r % gm) * 128);
     n0 = static_cast<int32_t>((r / gm) * BN);
   }
-  // symmetric products: each 128-column block of the tile below the diagonal
-  // is also written mirrored, the diagonal block as it is, and a block above
-  // the diagonal (in a 256-column tile on the diagonal) not at all: its
-  // mirror image comes from the tile below
-  const int32_t ti = m0 / 128;
+}
+
+template <int B_MN, int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                   const GemmTcArgs a) {
+  constexpr int kStages = gemm_stages<BN>();
+  constexpr uint32_t kStageBytes = stage_bytes<BN>();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + kStages * kStageBytes);
+  uint64_t *empty = full + kStages;
+  uint64_t *acc_full = empty + kStages;    // [2] accumulator b holds a finished tile
+  uint64_t *acc_empty = acc_full + 2;      // [2] accumulator b drained by the epilogue
+  uint64_t *done = acc_empty + 2;          // every MMA issued has completed
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = static_cast<int>(a.K / 64);
 
   if (threadIdx.x == 0) {
@@ -441,13 +453,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, 8);   // one arrival per epilogue warp
+    }
     mbar_init(done, 1);
     fence_mbar_init();
     tma_prefetch_desc(&mapA);
     tma_prefetch_desc(&mapB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -456,44 +472,73 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kStages;
-      if (kb >= kStages && !mbar_wait(empty + s, ((kb / kStages) - 1) & 1, a.status)) break;
-      uint8_t *As = sm + s * kStageBytes, *Bs = As + kStageA;
-      mbar_arrive_expect_tx(full + s, kStageBytes);
-      tma_load_3d(As, &mapA, kb * 64, m0, z, full + s);
-      if (B_MN) {   // BN / 64 boxes of 64 columns x 64 k-rows
+    // producer: k-block `it` (counted over all of this CTA's tiles) uses stage it % kStages
+    int64_t it = 0;
+    bool ok = true;
+    for (int64_t idx = blockIdx.x; idx < a.n_tiles && ok; idx += gridDim.x) {
+      int32_t m0, n0, z;
+      gemm_tile<BN>(a, idx, m0, n0, z);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = static_cast<int>(it % kStages);
+        const int64_t use = it / kStages;
+        if (use > 0 && !(ok = mbar_wait(empty + s, static_cast<uint32_t>((use - 1) & 1), a.status))) break;
+        uint8_t *As = sm + s * kStageBytes, *Bs = As + kStageA;
+        mbar_arrive_expect_tx(full + s, kStageBytes);
+        tma_load_3d(As, &mapA, kb * 64, m0, z, full + s);
+        if (B_MN) {   // BN / 64 boxes of 64 columns x 64 k-rows
 #pragma unroll
-        for (int j = 0; j < BN / 64; ++j) tma_load_3d(Bs + 8192 * j, &mapB, n0 + 64 * j, kb * 64, z, full + s);
-      } else {      // one box of 64 k-columns x BN rows
-        tma_load_3d(Bs, &mapB, kb * 64, n0, z, full + s);
+          for (int j = 0; j < BN / 64; ++j) tma_load_3d(Bs + 8192 * j, &mapB, n0 + 64 * j, kb * 64, z, full + s);
+        } else {      // one box of 64 k-columns x BN rows
+          tma_load_3d(Bs, &mapB, kb * 64, n0, z, full + s);
+        }
       }
     }
   } else if (warp == 1 && lane == 0) {
+    // MMA issuer: tile j of this CTA accumulates in TMEM columns (j % 2) * BN ..
+    int64_t it = 0, j = 0;
     bool ok = true;
-    for (int kb = 0; kb < nk && ok; ++kb) {
-      const int s = kb % kStages;
-      if (!(ok = mbar_wait(full + s, (kb / kStages) & 1, a.status))) break;
+    for (int64_t idx = blockIdx.x; idx < a.n_tiles && ok; idx += gridDim.x, ++j) {
+      const int b = static_cast<int>(j & 1);
+      if (j >= 2 && !(ok = mbar_wait(acc_empty + b, static_cast<uint32_t>(((j >> 1) - 1) & 1), a.status))) break;
       tc_fence_after();
-      const uint32_t as = smem_u32(sm + s * kStageBytes), bs = as + kStageA;
+      const uint32_t d = tmem + static_cast<uint32_t>(b * BN);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = static_cast<int>(it % kStages);
+        if (!(ok = mbar_wait(full + s, static_cast<uint32_t>((it / kStages) & 1), a.status))) break;
+        tc_fence_after();
+        const uint32_t as = smem_u32(sm + s * kStageBytes), bs = as + kStageA;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = sw128_desc(as + kk * 32, 16, 1024);
-        const uint64_t bd = B_MN ? sw128_desc(bs + kk * 2048, 8192, 1024) : sw128_desc(bs + kk * 32, 16, 1024);
-        mma_ss(tmem, ad, bd, a.idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = sw128_desc(as + kk * 32, 16, 1024);
+          const uint64_t bd = B_MN ? sw128_desc(bs + kk * 2048, 8192, 1024) : sw128_desc(bs + kk * 32, 16, 1024);
+          mma_ss(d, ad, bd, a.idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(empty + s);   // the stage is free once these MMAs have read it
       }
-      mma_commit(empty + s);
+      if (ok) mma_commit(acc_full + b);
     }
     mma_commit(done);
+    mbar_wait(done, 0, a.status);   // nothing of this CTA's is in flight when TMEM is released
   } else if (warp >= 2) {
-    const int q = warp & 3;
+    // epilogue: symmetric products write each 128-column block below the
+    // diagonal also mirrored, the diagonal block as it is, and a block above
+    // the diagonal (in a 256-column tile on the diagonal) not at all: its
+    // mirror image comes from the tile below
+    const int q = warp & 3;                    // TMEM lanes 32 q .. 32 q + 31
+    const int half = (warp - 2) >> 2;          // columns half * BN / 2 ..
     const int row = q * 32 + lane;
-    if (mbar_wait(done, 0, a.status)) {
+    int64_t j = 0;
+    for (int64_t idx = blockIdx.x; idx < a.n_tiles; idx += gridDim.x, ++j) {
+      const int b = static_cast<int>(j & 1);
+      if (!mbar_wait(acc_full + b, static_cast<uint32_t>((j >> 1) & 1), a.status)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      int32_t m0, n0, z;
+      gemm_tile<BN>(a, idx, m0, n0, z);
+      const int32_t ti = m0 / 128;
+      const uint32_t taddr = tmem + static_cast<uint32_t>(b * BN) + (static_cast<uint32_t>(q * 32) << 16);
       const int64_t obase = z * a.ep.stride + static_cast<int64_t>(m0 + row) * a.ep.N + n0;
 #pragma unroll 1
-      for (int i = 0; i < BN / 32; ++i) {
+      for (int i = half * (BN / 64); i < (half + 1) * (BN / 64); ++i) {
         const int32_t ct = (n0 + 32 * i) / 128;   // 128-column block of the output
         if (a.ep.sym && ct > ti) break;          // above the diagonal (the tile's last block)
         const bool mirror = a.ep.sym && ct < ti;
@@ -501,12 +546,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld32(taddr + 32 * i, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int64_t col = n0 + 32 * i + 8 * j;
-          epi_store8(a.ep, obase + 32 * i + 8 * j, m0 + row, col, v + 8 * j, mirror,
+        for (int jj = 0; jj < 4; ++jj) {
+          const int64_t col = n0 + 32 * i + 8 * jj;
+          epi_store8(a.ep, obase + 32 * i + 8 * jj, m0 + row, col, v + 8 * jj, mirror,
                      z * a.ep.stride + col * a.ep.N + m0 + row);
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + b);
     }
   }
   tc_fence_before();
@@ -514,7 +562,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -648,13 +696,21 @@ cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int6
     if (!make_batch_map(&mb, B, batch, 64, 64)) return cudaErrorInvalidValue;
   }
   a.idesc = idesc_f16(128, static_cast<uint32_t>(BN), A.dtype == HIMUON_FP16 ? 0u : 1u, 0, b_trans ? 0u : 1u, 0);
-  dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(M / 128), static_cast<unsigned>(batch));
-  if (a.ep.sym) {   // the tiles reaching the lower triangle (see the kernel)
+  a.gx = static_cast<int32_t>(N / BN);
+  a.gy = static_cast<int32_t>(M / 128);
+  if (a.ep.sym) {   // the tiles reaching the lower triangle (see gemm_tile)
     const int64_t nt = M / 128;
     int64_t count = 0;
     for (int64_t ti = 0; ti < nt; ++ti) count += BN == 128 ? ti + 1 : ti / 2 + 1;
-    grid = dim3(static_cast<unsigned>(count), 1, static_cast<unsigned>(batch));
+    a.tiles_per_matrix = count;
+  } else {
+    a.tiles_per_matrix = static_cast<int64_t>(a.gx) * a.gy;
   }
+  a.n_tiles = a.tiles_per_matrix * batch;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(a.n_tiles, sms)));
   cudaError_t e;
   auto go = [&](auto kern, uint32_t smem) -> cudaError_t {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -663,16 +719,8 @@ cudaError_t gemm_tc(const Batch &A, const Batch &B, int b_trans, int64_t M, int6
     kern<<<grid, kGemmThreads, smem, stream>>>(ma, mb, a);
     return cudaSuccess;
   };
-  const bool short_k = K <= 256;
-  if (BN == 256) {
-    // two stages (97 KB): two CTAs share an SM, so one's epilogue overlaps the
-    // other's main loop (three stages, one CTA per SM, ran 6% slower)
-    if (b_trans) e = go(gemm_tc_kernel<0, 2, 256>, gemm_smem<2, 256>());
-    else e = go(gemm_tc_kernel<1, 2, 256>, gemm_smem<2, 256>());
-  } else {
-    if (b_trans) e = short_k ? go(gemm_tc_kernel<0, 2, 128>, gemm_smem<2, 128>()) : go(gemm_tc_kernel<0, 3, 128>, gemm_smem<3, 128>());
-    else e = short_k ? go(gemm_tc_kernel<1, 2, 128>, gemm_smem<2, 128>()) : go(gemm_tc_kernel<1, 3, 128>, gemm_smem<3, 128>());
-  }
+  if (BN == 256) e = b_trans ? go(gemm_tc_kernel<0, 256>, gemm_smem<256>()) : go(gemm_tc_kernel<1, 256>, gemm_smem<256>());
+  else e = b_trans ? go(gemm_tc_kernel<0, 128>, gemm_smem<128>()) : go(gemm_tc_kernel<1, 128>, gemm_smem<128>());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
