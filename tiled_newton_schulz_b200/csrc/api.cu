@@ -598,6 +598,7 @@ Epilogue epi(float alpha, float beta, const float *c32, float *out32, void *out1
   e.out2_16 = nullptr;
   e.diag2 = 0.f;
   e.sym = 0;
+  e.lower32 = 0;
   return e;
 }
 Epilogue sym(Epilogue e) {
@@ -724,12 +725,19 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
         auto rzop = [&]() -> void * { return f32 ? static_cast<void *>(rz32) : rz16; };
         auto qop = [&](int i) -> void * { return f32 ? static_cast<void *>(qf[i]) : q16[i]; };
         bool q_identity = true;
+        // every fp32 n x n matrix here is read only as the C term of another
+        // symmetric product: its blocks above the diagonal are never written
+        auto gsym = [f32](Epilogue e) {
+          e.sym = 1;
+          e.lower32 = f32 ? 0 : 1;
+          return e;
+        };
         auto restarts_at = [&p](int t) {
           for (int i = 0; i < p.n_restart; ++i)
             if (p.restart_at[i] == t) return true;
           return false;
         };
-        rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, sym(epi(1.f, 0.f, nullptr, r32, r16, dt16)));
+        rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, gsym(epi(1.f, 0.f, nullptr, r32, r16, dt16)));
         for (int t = 1; t <= p.steps && rc == HIMUON_OK; ++t) {
           const float a = p.coeffs[3 * (t - 1)], b = p.coeffs[3 * (t - 1) + 1], cc = p.coeffs[3 * (t - 1) + 2];
           const bool restart = restarts_at(t);
@@ -749,14 +757,14 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
                 cur = 1 - cur;
               }
               if (rc) break;
-              rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, sym(epi(1.f, 0.f, nullptr, r32, r16, dt16)));
+              rc = ops.mm(xop(cur), n, m, xop(cur), n, m, 1, n, n, m, bc, gsym(epi(1.f, 0.f, nullptr, r32, r16, dt16)));
               if (rc) break;
             }
             q_identity = true;
           }
           // Z = b R + c R^2 (fp32 copy only when the operands are fp32).  Right
           // after Q = I the same epilogue also writes Q <- Q Z + a Q = Z + a I.
-          Epilogue ez = sym(epi(cc, b, r32, f32 ? z32 : nullptr, z16, dt16));
+          Epilogue ez = gsym(epi(cc, b, r32, f32 ? z32 : nullptr, z16, dt16));
           if (q_identity) {
             ez.out2_32 = qf[qc];
             ez.out2_16 = f32 ? nullptr : q16[qc];
@@ -769,17 +777,17 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
             q_identity = false;
           } else {
             rc = ops.mm(qop(qc), n, n, zop(), n, n, 0, n, n, n, bc,
-                        sym(epi(1.f, a, qf[qc], (f32 || !last_use) ? qf[1 - qc] : nullptr,
+                        gsym(epi(1.f, a, qf[qc], (f32 || !last_use) ? qf[1 - qc] : nullptr,
                                 f32 ? nullptr : q16[1 - qc], dt16)));
             qc = 1 - qc;
             if (rc) break;
           }
           if (last_use) continue;   // R_K, and R before a restart, are never used
           // RZ <- R Z + a R
-          rc = ops.mm(rop(), n, n, zop(), n, n, 0, n, n, n, bc, sym(epi(1.f, a, r32, rz32, rz16, dt16)));
+          rc = ops.mm(rop(), n, n, zop(), n, n, 0, n, n, n, bc, gsym(epi(1.f, a, r32, rz32, rz16, dt16)));
           if (rc) break;
           // R <- Z RZ + a RZ
-          rc = ops.mm(zop(), n, n, rzop(), n, n, 0, n, n, n, bc, sym(epi(1.f, a, rz32, r32, r16, dt16)));
+          rc = ops.mm(zop(), n, n, rzop(), n, n, 0, n, n, n, bc, gsym(epi(1.f, a, rz32, r32, r16, dt16)));
         }
         if (rc == HIMUON_OK) {
           // output Q X

@@ -268,6 +268,7 @@ struct EpiArgs {
   void *out2_16;
   float diag2;
   int32_t sym;      // lower-triangle tiles only, off-diagonal ones mirrored
+  int32_t lower32;  // with sym: no mirrored copies in the fp32 outputs
   int64_t N;        // columns of the output matrices
   int64_t stride;   // elements per output matrix (M * N)
 };
@@ -279,7 +280,7 @@ __device__ __forceinline__ void epi_put8(const EpiArgs &e, float *out32, void *o
   if (out32) {
     *reinterpret_cast<float4 *>(out32 + o) = make_float4(v[0], v[1], v[2], v[3]);
     *reinterpret_cast<float4 *>(out32 + o + 4) = make_float4(v[4], v[5], v[6], v[7]);
-    if (mirror) {
+    if (mirror && !e.lower32) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) out32[om + i * e.N] = v[i];
     }
@@ -670,6 +671,7 @@ EpiArgs to_epi(const Epilogue &e, int64_t M, int64_t N) {
   a.out2_16 = e.out2_16;
   a.diag2 = e.diag2;
   a.sym = e.sym && M == N;
+  a.lower32 = a.sym && e.lower32;
   a.N = N;
   a.stride = M * N;
   return a;

@@ -38,6 +38,11 @@ struct Epilogue {
   // tensor-core version computes only the 128 x 128 tiles on and below the
   // diagonal and writes each off-diagonal one twice, mirrored.
   int32_t sym;
+  // With sym: the fp32 outputs (out32, out2_32) get only the 128 x 128 blocks
+  // on and below the diagonal, not the mirrored copies above it (for a
+  // matrix read only as the C term of other symmetric products, which read
+  // those blocks alone).  The 16-bit outputs, read as operands, stay whole.
+  int32_t lower32;
 };
 
 // acc = A * B^T (b_trans = 1, B is N x K) or A * B (b_trans = 0, B is K x N),
