@@ -209,6 +209,38 @@ def test_full_ns_bf16_with_transpose(hm, H, W):
     check16(y, oracle.ns_map(xin, C32), 0)
 
 
+@pytest.mark.parametrize("dtype", ["float32", "float16"])
+@pytest.mark.parametrize("H,W,T", [(300, 700, 0), (700, 300, 0), (600, 520, 512), (520, 600, 512)])
+def test_staged_16bit_compute_io_dtypes(hm, H, W, T, dtype):
+    """16-bit operands with fp32 or fp16 inputs and outputs on the staged path,
+    whose last product writes the caller's buffer from its epilogue: straight
+    and transposed tiles, ragged edges (600 x 520 at T = 512 has 88-wide and
+    88-high tiles)."""
+    X = inputs.gaussian((H, W), seed=H + 5 * W + T)
+    xin, y = run_ns(hm, X, T, hm.BF16, getattr(torch, dtype), full=T == 0)
+    ref = oracle.ns_map(xin, C32) if T == 0 else oracle.ns_tiled(xin, T, C32)
+    check16(y, ref, T)
+
+
+def test_staged_momentum_step_fp32_w_and_update_out(hm):
+    """The staged momentum step (T = 512, ragged and transposed tiles) with an
+    fp32 W and a bf16 update output: O matches the oracle per tile and
+    W' = W - lr O within lr times O's tolerance (fp32 W adds no rounding of
+    note)."""
+    H, W, T, lr = 700, 600, 512, 0.02
+    w0 = 0.02 * inputs.gaussian((H, W), seed=11)
+    m0 = inputs.low_rank_plus_noise(H, W, inputs.sigma_inverse(16), 0.01, seed=12)
+    g0 = inputs.low_rank_plus_noise(H, W, inputs.sigma_inverse(16), 0.01, seed=13)
+    w, m, g = dev(w0, torch.float32), dev(m0, torch.bfloat16), dev(g0, torch.bfloat16)
+    o = torch.empty_like(m)
+    mi, gi, wi = to_np(m), to_np(g), to_np(w)
+    hm.momentum_step([w], [m], [g], 0.95, lr, hm.params(T, QUINTIC, steps=5), update_out=[o])
+    assert hm.device_status() == 0
+    W2, _, O = oracle.momentum_step(wi, mi, gi, 0.95, lr, T, C32)
+    check16(to_np(o), O, T)
+    assert np.linalg.norm(to_np(w) - W2) <= float(np.float32(lr)) * TOL16 * np.linalg.norm(O)
+
+
 def test_momentum_step_resident(hm):
     shapes = [(256, 256), (256, 512), (384, 128)]
     rng = np.random.default_rng(12)

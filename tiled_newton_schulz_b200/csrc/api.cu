@@ -599,6 +599,10 @@ Epilogue epi(float alpha, float beta, const float *c32, float *out32, void *out1
   e.diag2 = 0.f;
   e.sym = 0;
   e.lower32 = 0;
+  e.sc_tiles = nullptr;
+  e.sc_blocks = nullptr;
+  e.sc_mode = 0;
+  e.sc_lr = 0.f;
   return e;
 }
 Epilogue sym(Epilogue e) {
@@ -670,6 +674,17 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       int rc = HIMUON_OK;
       // operand views: fp32 path reads the fp32 buffers directly
       auto xop = [&](int i) -> void * { return f32 ? static_cast<void *>(x32[i]) : x16[i]; };
+      // the last product of the 16-bit paths writes the blocks' roles itself
+      // (no fp32 copy of the result and no unpack pass)
+      auto scatter = [&](Epilogue e) {
+        e.out32 = nullptr;
+        e.out16 = nullptr;
+        e.sc_tiles = tiles;
+        e.sc_blocks = plan.d_blocks;
+        e.sc_mode = step ? 1 : 0;
+        e.sc_lr = lr;
+        return e;
+      };
       if (!gram) {
         void *bop = f32 ? static_cast<void *>(W + L.b32) : W + L.b16;
         for (int t = 0; t < p.steps && rc == HIMUON_OK; ++t) {
@@ -700,7 +715,8 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
             // the 16-bit operand for the next step, or the fp32 result after the last
             // (step 0 of the bf16 path: Bop (X / rho) = (Bop X) / rho)
             const bool last = t + 1 == p.steps;
-            Epilogue e3 = epi(1.f, 0.f, nullptr, last ? x32[0] : nullptr, last ? nullptr : x16[1 - cur], dt16);
+            Epilogue e3 = epi(1.f, 0.f, nullptr, nullptr, x16[1 - cur], dt16);
+            if (last) e3 = scatter(e3);
             if (prescale && t == 0) e3.alpha_batch = inv;
             rc = ops.mm(bop, n, n, x16[cur], n, m, 0, n, m, n, bc, e3);
             cur = 1 - cur;
@@ -795,11 +811,12 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
             rc = ops.mm(qop(qc), n, n, x32[cur], n, m, 0, n, m, n, bc, epi(1.f, 0.f, nullptr, x32[1 - cur], nullptr, dt16));
             xfinal = x32[1 - cur];
           } else {
-            rc = ops.mm(qop(qc), n, n, x16[cur], n, m, 0, n, m, n, bc, epi(1.f, 0.f, nullptr, x32[0], nullptr, dt16));
+            rc = ops.mm(qop(qc), n, n, x16[cur], n, m, 0, n, m, n, bc, scatter(epi(1.f, 0.f, nullptr, nullptr, nullptr, dt16)));
           }
         }
       }
       if (rc) return rc;
+      if (!f32) continue;   // written by the last product's epilogue
       UnpackArgs ua;
       ua.blocks = plan.d_blocks;
       ua.tiles = tiles;

@@ -269,6 +269,10 @@ struct EpiArgs {
   float diag2;
   int32_t sym;      // lower-triangle tiles only, off-diagonal ones mirrored
   int32_t lower32;  // with sym: no mirrored copies in the fp32 outputs
+  const DevTile *sc_tiles;   // scatter to the blocks' roles (nullptr: out32/out16)
+  const DevBlock *sc_blocks;
+  int32_t sc_mode;
+  float sc_lr;
   int64_t N;        // columns of the output matrices
   int64_t stride;   // elements per output matrix (M * N)
 };
@@ -303,6 +307,53 @@ __device__ __forceinline__ void epi_put8(const EpiArgs &e, float *out32, void *o
       uint16_t *d = static_cast<uint16_t *>(out16);
 #pragma unroll
       for (int i = 0; i < 8; ++i) d[om + i * e.N] = hs[i];
+    }
+  }
+}
+
+// Scatter 8 values of matrix z (row `row`, columns col..col+7 of the n x m
+// tile operand) to the block they came from: the unpack pass's element map.
+// Straight tiles write a run of a block row (one 16-byte access per role
+// where the alignment allows); transposed ones write column c0 + row of the
+// block, one element per row col..col+7 (a warp's lanes hold consecutive
+// rows, so each of these stores is coalesced).
+__device__ __forceinline__ void epi_scatter8(const EpiArgs &e, int64_t z, int64_t row, int64_t col, const float (&v)[8]) {
+  const DevTile tl = e.sc_tiles[z];
+  const DevBlock &b = e.sc_blocks[tl.block];
+  void *out = b.ptr[kRoleOut];
+  void *wp = e.sc_mode == 1 ? b.ptr[kRoleW] : nullptr;
+  const int32_t dto = b.dtype[kRoleOut], dtw = b.dtype[kRoleW];
+  const int64_t ldo = b.ld[kRoleOut], ldw = b.ld[kRoleW];
+  if (!tl.transposed) {
+    if (row >= tl.h || col >= tl.w) return;   // zero padding of a ragged tile
+    const int64_t r = tl.r0 + row, c = tl.c0 + col;
+    if (col + 8 <= tl.w && (!out || vec8_ok(out, dto, ldo, static_cast<int32_t>(c))) &&
+        (!wp || vec8_ok(wp, dtw, ldw, static_cast<int32_t>(c)))) {
+      if (out) st8_16(out, dto, r * ldo + c, v);
+      if (wp) {
+        float w[8];
+        ld8_16(wp, dtw, r * ldw + c, w);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = fmaf(-e.sc_lr, v[i], w[i]);
+        st8_16(wp, dtw, r * ldw + c, w);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (col + i >= tl.w) break;
+        if (out) st_elem(out, dto, r * ldo + c + i, v[i]);
+        if (wp) st_elem(wp, dtw, r * ldw + c + i, fmaf(-e.sc_lr, v[i], ld_elem(wp, dtw, r * ldw + c + i)));
+      }
+    }
+  } else {
+    if (row >= tl.w) return;   // operand row `row` is block column c0 + row
+    const int64_t c = tl.c0 + row;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (col + i >= tl.h) break;
+      const int64_t r = tl.r0 + col + i;
+      if (out) st_elem(out, dto, r * ldo + c, v[i]);
+      if (wp) st_elem(wp, dtw, r * ldw + c, fmaf(-e.sc_lr, v[i], ld_elem(wp, dtw, r * ldw + c)));
     }
   }
 }
@@ -352,6 +403,10 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
   if (e.diag != 0.f && on_diag) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] += (col + i == row) ? e.diag : 0.f;
+  }
+  if (e.sc_tiles) {
+    epi_scatter8(e, o / e.stride, row, col, v);
+    return;
   }
   epi_put8(e, e.out32, e.out16, o, v, mirror, om);
   if (e.out2_32 || e.out2_16) {
@@ -672,6 +727,10 @@ EpiArgs to_epi(const Epilogue &e, int64_t M, int64_t N) {
   a.diag2 = e.diag2;
   a.sym = e.sym && M == N;
   a.lower32 = a.sym && e.lower32;
+  a.sc_tiles = e.sc_tiles;
+  a.sc_blocks = e.sc_blocks;
+  a.sc_mode = e.sc_mode;
+  a.sc_lr = e.sc_lr;
   a.N = N;
   a.stride = M * N;
   return a;

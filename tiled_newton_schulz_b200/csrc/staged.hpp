@@ -43,6 +43,14 @@ struct Epilogue {
   // matrix read only as the C term of other symmetric products, which read
   // those blocks alone).  The 16-bit outputs, read as operands, stay whole.
   int32_t lower32;
+  // Scatter (tensor-core path): instead of out32/out16, matrix z of the batch
+  // is the tile sc_tiles[z]; its valid h x w part (transposed back when the
+  // tile is) goes straight to its block's Out role and, with sc_mode 1, into
+  // W -= sc_lr * O, as launch_unpack would write it from an fp32 copy.
+  const DevTile *sc_tiles;
+  const DevBlock *sc_blocks;
+  int32_t sc_mode;
+  float sc_lr;
 };
 
 // acc = A * B^T (b_trans = 1, B is N x K) or A * B (b_trans = 0, B is K x N),
