@@ -96,7 +96,7 @@ def test_workspace_size_on_the_host(lib):
     assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p256f), 0) > 0    # fp32: staged
     p512 = himuon.params(512, (3.4445, -4.7750, 2.0315), steps=5)
     need = lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p512), 0)
-    assert need > 512 * 512 * 4 * 64                        # at least the fp32 iterate of the 64 tiles
+    assert need > 512 * 512 * 4 * 64                        # at least the two 16-bit iterates of the 64 tiles
     pc = himuon.params(512, (3.4445, -4.7750, 2.0315), steps=5, chunk_bytes=64 << 20)
     assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(pc), 0) <= 64 << 20
 

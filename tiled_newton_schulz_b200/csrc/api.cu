@@ -499,7 +499,10 @@ WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, bool gram) 
   };
   const size_t nm = static_cast<size_t>(n * m * count), nn = static_cast<size_t>(n * n * count);
   const bool f32 = compute == HIMUON_FP32;
-  L.x32a = take(4 * nm);
+  // fp32 X: the fp32 path's iterate, and the input the normalisation pass
+  // reads (fp16 operands and Gram NS).  bf16 NS packs straight to 16 bits and
+  // its last product writes the caller's buffers: it needs none.
+  if (f32 || gram || compute != HIMUON_BF16) L.x32a = take(4 * nm);
   if (f32) L.x32b = take(4 * nm);
   else {
     L.x16a = take(2 * nm);

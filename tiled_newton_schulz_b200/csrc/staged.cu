@@ -311,49 +311,72 @@ __device__ __forceinline__ void epi_put8(const EpiArgs &e, float *out32, void *o
   }
 }
 
-// Scatter 8 values of matrix z (row `row`, columns col..col+7 of the n x m
-// tile operand) to the block they came from: the unpack pass's element map.
-// Straight tiles write a run of a block row (one 16-byte access per role
-// where the alignment allows); transposed ones write column c0 + row of the
-// block, one element per row col..col+7 (a warp's lanes hold consecutive
-// rows, so each of these stores is coalesced).
-__device__ __forceinline__ void epi_scatter8(const EpiArgs &e, int64_t z, int64_t row, int64_t col, const float (&v)[8]) {
+// Where the scatter epilogue puts matrix z of the batch: its tile's block
+// roles, resolved once per output tile.
+struct ScatterDst {
+  void *out, *w;
+  int64_t ldo, ldw;
+  int32_t dto, dtw;
+  int32_t r0, c0, h, wd, transposed;
+  bool vec;   // 16-byte runs allowed for every role written
+};
+
+__device__ __forceinline__ ScatterDst scatter_dst(const EpiArgs &e, int64_t z) {
   const DevTile tl = e.sc_tiles[z];
   const DevBlock &b = e.sc_blocks[tl.block];
-  void *out = b.ptr[kRoleOut];
-  void *wp = e.sc_mode == 1 ? b.ptr[kRoleW] : nullptr;
-  const int32_t dto = b.dtype[kRoleOut], dtw = b.dtype[kRoleW];
-  const int64_t ldo = b.ld[kRoleOut], ldw = b.ld[kRoleW];
-  if (!tl.transposed) {
-    if (row >= tl.h || col >= tl.w) return;   // zero padding of a ragged tile
-    const int64_t r = tl.r0 + row, c = tl.c0 + col;
-    if (col + 8 <= tl.w && (!out || vec8_ok(out, dto, ldo, static_cast<int32_t>(c))) &&
-        (!wp || vec8_ok(wp, dtw, ldw, static_cast<int32_t>(c)))) {
-      if (out) st8_16(out, dto, r * ldo + c, v);
-      if (wp) {
+  ScatterDst d;
+  d.out = b.ptr[kRoleOut];
+  d.w = e.sc_mode == 1 ? b.ptr[kRoleW] : nullptr;
+  d.ldo = b.ld[kRoleOut];
+  d.ldw = b.ld[kRoleW];
+  d.dto = b.dtype[kRoleOut];
+  d.dtw = b.dtype[kRoleW];
+  d.r0 = tl.r0;
+  d.c0 = tl.c0;
+  d.h = tl.h;
+  d.wd = tl.w;
+  d.transposed = tl.transposed;
+  d.vec = (!d.out || vec8_ok(d.out, d.dto, d.ldo, tl.c0)) && (!d.w || vec8_ok(d.w, d.dtw, d.ldw, tl.c0));
+  return d;
+}
+
+// Scatter 8 values (row `row`, columns col..col+7 of the n x m tile operand)
+// to the block they came from: the unpack pass's element map.  Straight
+// tiles write a run of a block row (one 16-byte access per role where the
+// alignment allows); transposed ones write column c0 + row of the block, one
+// element per row col..col+7 (a warp's lanes hold consecutive rows, so each
+// of these stores is coalesced).
+__device__ __forceinline__ void epi_scatter8(const EpiArgs &e, const ScatterDst &d, int64_t row, int64_t col,
+                                             const float (&v)[8]) {
+  if (!d.transposed) {
+    if (row >= d.h || col >= d.wd) return;   // zero padding of a ragged tile
+    const int64_t r = d.r0 + row, c = d.c0 + col;
+    if (col + 8 <= d.wd && d.vec) {
+      if (d.out) st8_16(d.out, d.dto, r * d.ldo + c, v);
+      if (d.w) {
         float w[8];
-        ld8_16(wp, dtw, r * ldw + c, w);
+        ld8_16(d.w, d.dtw, r * d.ldw + c, w);
 #pragma unroll
         for (int i = 0; i < 8; ++i) w[i] = fmaf(-e.sc_lr, v[i], w[i]);
-        st8_16(wp, dtw, r * ldw + c, w);
+        st8_16(d.w, d.dtw, r * d.ldw + c, w);
       }
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        if (col + i >= tl.w) break;
-        if (out) st_elem(out, dto, r * ldo + c + i, v[i]);
-        if (wp) st_elem(wp, dtw, r * ldw + c + i, fmaf(-e.sc_lr, v[i], ld_elem(wp, dtw, r * ldw + c + i)));
+        if (col + i >= d.wd) break;
+        if (d.out) st_elem(d.out, d.dto, r * d.ldo + c + i, v[i]);
+        if (d.w) st_elem(d.w, d.dtw, r * d.ldw + c + i, fmaf(-e.sc_lr, v[i], ld_elem(d.w, d.dtw, r * d.ldw + c + i)));
       }
     }
   } else {
-    if (row >= tl.w) return;   // operand row `row` is block column c0 + row
-    const int64_t c = tl.c0 + row;
+    if (row >= d.wd) return;   // operand row `row` is block column c0 + row
+    const int64_t c = d.c0 + row;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      if (col + i >= tl.h) break;
-      const int64_t r = tl.r0 + col + i;
-      if (out) st_elem(out, dto, r * ldo + c, v[i]);
-      if (wp) st_elem(wp, dtw, r * ldw + c, fmaf(-e.sc_lr, v[i], ld_elem(wp, dtw, r * ldw + c)));
+      if (col + i >= d.h) break;
+      const int64_t r = d.r0 + col + i;
+      if (d.out) st_elem(d.out, d.dto, r * d.ldo + c, v[i]);
+      if (d.w) st_elem(d.w, d.dtw, r * d.ldw + c, fmaf(-e.sc_lr, v[i], ld_elem(d.w, d.dtw, r * d.ldw + c)));
     }
   }
 }
@@ -363,9 +386,10 @@ __device__ __forceinline__ void epi_scatter8(const EpiArgs &e, int64_t z, int64_
 // (an off-diagonal tile of a symmetric product) they also go to rows
 // col..col+7, column `row` (element index `om` for the first; a warp's lanes
 // hold consecutive rows, so each of these scalar stores is coalesced).
+// `alpha` is the product's alpha for this matrix and `sd`, with the scatter
+// epilogue, its destination (both resolved once per output tile).
 __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t row, int64_t col, const float *acc,
-                                           bool mirror = false, int64_t om = 0) {
-  const float alpha = e.alpha_batch ? e.alpha_batch[o / e.stride] : e.alpha;
+                                           bool mirror, int64_t om, float alpha, const ScatterDst &sd) {
   float v[8];
   if (e.c32) {
     const float4 c0 = *reinterpret_cast<const float4 *>(e.c32 + o);
@@ -405,7 +429,7 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
     for (int i = 0; i < 8; ++i) v[i] += (col + i == row) ? e.diag : 0.f;
   }
   if (e.sc_tiles) {
-    epi_scatter8(e, o / e.stride, row, col, v);
+    epi_scatter8(e, sd, row, col, v);
     return;
   }
   epi_put8(e, e.out32, e.out16, o, v, mirror, om);
@@ -591,6 +615,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int32_t m0, n0, z;
       gemm_tile<BN>(a, idx, m0, n0, z);
       const int32_t ti = m0 / 128;
+      const float alpha = a.ep.alpha_batch ? a.ep.alpha_batch[z] : a.ep.alpha;
+      ScatterDst sd{};
+      if (a.ep.sc_tiles) sd = scatter_dst(a.ep, z);
       const uint32_t taddr = tmem + static_cast<uint32_t>(b * BN) + (static_cast<uint32_t>(q * 32) << 16);
       const int64_t obase = z * a.ep.stride + static_cast<int64_t>(m0 + row) * a.ep.N + n0;
 #pragma unroll 1
@@ -605,7 +632,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int jj = 0; jj < 4; ++jj) {
           const int64_t col = n0 + 32 * i + 8 * jj;
           epi_store8(a.ep, obase + 32 * i + 8 * jj, m0 + row, col, v + 8 * jj, mirror,
-                     z * a.ep.stride + col * a.ep.N + m0 + row);
+                     z * a.ep.stride + col * a.ep.N + m0 + row, alpha, sd);
         }
       }
       tc_fence_before();
