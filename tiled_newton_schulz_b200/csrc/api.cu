@@ -514,11 +514,14 @@ WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, bool gram) 
     if (f32) L.b32 = take(4 * nn);
     else L.b16 = take(2 * nn);
   } else {
-    L.q32 = take(4 * nn);
-    L.z32 = take(4 * nn);
+    // fp32 R (a32) and RZ in both arithmetics (C terms); Q and Z in fp32 only
+    // when they are the operands
     L.rz32 = take(4 * nn);
-    if (f32) L.b32 = take(4 * nn);   // second Q buffer
-    else {
+    if (f32) {
+      L.q32 = take(4 * nn);
+      L.z32 = take(4 * nn);
+      L.b32 = take(4 * nn);   // second Q buffer
+    } else {
       L.q16a = take(2 * nn);
       L.q16b = take(2 * nn);
       L.z16 = take(2 * nn);
@@ -727,8 +730,14 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
         }
       } else {
         // Gram NS (Algorithm 3): R = X X^T, Q = I; restarts X <- Q X.  The terms
-        // a Q, a R, a RZ stay fp32 (C operands): folding a I into a 16-bit Z
-        // loses R's small eigen-directions below fp16's normal range.  Between
+        // a R, a RZ stay fp32 (C operands): folding a I into a 16-bit Z, or
+        // reading R or RZ rounded to 16 bits, loses R's small eigen-directions
+        // (below fp16's normal range), which later steps feed back (fp16 R and
+        // RZ terms: 4.6% error on a 256 x 1024 input without a restart).  The
+        // a Q term reads the 16-bit Q: Q's eigenvalues stay of the order of a
+        // or above and Q is never fed back into R, so its rounding costs
+        // nothing (equal or smaller errors under every restart pattern tried,
+        // in an fp16 emulation against the fp64 map).  Between
         // restarts every n x n matrix here is a polynomial in one R, so all of
         // them commute and every n x n product is symmetric: computed as its
         // lower triangle.
@@ -737,7 +746,7 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
         float *q32b = f32 ? reinterpret_cast<float *>(W + L.b32) : nullptr;
         void *r16 = a16, *z16 = f32 ? nullptr : W + L.z16, *rz16 = f32 ? nullptr : W + L.rz16;
         void *q16[2] = {f32 ? nullptr : W + L.q16a, f32 ? nullptr : W + L.q16b};
-        float *qf[2] = {q32, f32 ? q32b : q32};
+        float *qf[2] = {f32 ? q32 : nullptr, q32b};   // fp32 Q: the fp32 path only
         int qc = 0;
         auto rop = [&]() -> void * { return f32 ? static_cast<void *>(r32) : r16; };
         auto zop = [&]() -> void * { return f32 ? static_cast<void *>(z32) : z16; };
@@ -785,7 +794,7 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
           // after Q = I the same epilogue also writes Q <- Q Z + a Q = Z + a I.
           Epilogue ez = gsym(epi(cc, b, r32, f32 ? z32 : nullptr, z16, dt16));
           if (q_identity) {
-            ez.out2_32 = qf[qc];
+            ez.out2_32 = f32 ? qf[qc] : nullptr;
             ez.out2_16 = f32 ? nullptr : q16[qc];
             ez.diag2 = a;
           }
@@ -795,9 +804,9 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
           if (q_identity) {
             q_identity = false;
           } else {
-            rc = ops.mm(qop(qc), n, n, zop(), n, n, 0, n, n, n, bc,
-                        gsym(epi(1.f, a, qf[qc], (f32 || !last_use) ? qf[1 - qc] : nullptr,
-                                f32 ? nullptr : q16[1 - qc], dt16)));
+            Epilogue eq = f32 ? epi(1.f, a, qf[qc], qf[1 - qc], nullptr, dt16) : epi(1.f, a, nullptr, nullptr, q16[1 - qc], dt16);
+            if (!f32) eq.c16 = q16[qc];
+            rc = ops.mm(qop(qc), n, n, zop(), n, n, 0, n, n, n, bc, gsym(eq));
             qc = 1 - qc;
             if (rc) break;
           }
