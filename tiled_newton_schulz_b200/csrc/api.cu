@@ -488,7 +488,18 @@ struct WsLayout {
   size_t x32a, x32b, x16a, x16b, a32, a16, b32, b16, q32, q16a, q16b, z32, z16, rz32, rz16, partial, scale, total;
 };
 
-WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, bool gram) {
+// The 16-bit element paths of one call: bf16 NS packs the input unscaled and
+// its first products apply 1/rho (prescale); other 16-bit calls without a
+// momentum update (fp16 NS, Gram NS) sum squares in one pass over the input
+// and write the scaled operand in a second (two_pass); the rest pack to fp32
+// and normalise from there.
+bool staged_prescale(int compute, int op) { return compute == HIMUON_BF16 && op != HIMUON_OP_GRAM_NS; }
+bool staged_two_pass(int compute, int op) {
+  return compute != HIMUON_FP32 && !staged_prescale(compute, op) && op != HIMUON_OP_MOMENTUM_STEP;
+}
+
+WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, int op) {
+  const bool gram = op == HIMUON_OP_GRAM_NS;
   WsLayout L;
   memset(&L, 0, sizeof L);
   size_t off = 0;
@@ -500,9 +511,9 @@ WsLayout ws_layout(int64_t n, int64_t m, int64_t count, int compute, bool gram) 
   const size_t nm = static_cast<size_t>(n * m * count), nn = static_cast<size_t>(n * n * count);
   const bool f32 = compute == HIMUON_FP32;
   // fp32 X: the fp32 path's iterate, and the input the normalisation pass
-  // reads (fp16 operands and Gram NS).  bf16 NS packs straight to 16 bits and
-  // its last product writes the caller's buffers: it needs none.
-  if (f32 || gram || compute != HIMUON_BF16) L.x32a = take(4 * nm);
+  // reads (the fp16 momentum step).  The other 16-bit paths pack straight to
+  // 16 bits and their last product writes the caller's buffers.
+  if (f32 || (!staged_prescale(compute, op) && !staged_two_pass(compute, op))) L.x32a = take(4 * nm);
   if (f32) L.x32b = take(4 * nm);
   else {
     L.x16a = take(2 * nm);
@@ -544,13 +555,13 @@ size_t chunk_limit(size_t ws_bytes, const himuon_ns_params &p) {
 // Tiles per chunk of a class under the limit (0 if even one tile does not fit):
 // the fewest chunks the limit allows, of equal size (a last chunk of a tile or
 // two would run every product of the call once more at a tiny batch).
-int64_t chunk_tiles(const TileClass &c, size_t limit, int compute, bool gram) {
+int64_t chunk_tiles(const TileClass &c, size_t limit, int compute, int op) {
   const int64_t tiles = static_cast<int64_t>(c.tiles.size());
-  if (tiles < 1 || ws_layout(c.n, c.m, 1, compute, gram).total > limit) return 0;
+  if (tiles < 1 || ws_layout(c.n, c.m, 1, compute, op).total > limit) return 0;
   int64_t lo = 1, hi = std::min<int64_t>(tiles, 65535);   // the workspace grows with the tile count
   while (lo < hi) {
     const int64_t mid = (lo + hi + 1) / 2;
-    if (ws_layout(c.n, c.m, mid, compute, gram).total <= limit) lo = mid;
+    if (ws_layout(c.n, c.m, mid, compute, op).total <= limit) lo = mid;
     else hi = mid - 1;
   }
   const int64_t chunks = (tiles + lo - 1) / lo;
@@ -558,11 +569,10 @@ int64_t chunk_tiles(const TileClass &c, size_t limit, int compute, bool gram) {
 }
 
 int64_t staged_ws_bytes(const Plan &plan, int op, int compute) {
-  const bool gram = op == HIMUON_OP_GRAM_NS;
   int64_t need = 0;
   for (const TileClass &c : plan.classes)
     need = std::max<int64_t>(need,
-                             static_cast<int64_t>(ws_layout(c.n, c.m, 1, class_compute(c, op, compute), gram).total));
+                             static_cast<int64_t>(ws_layout(c.n, c.m, 1, class_compute(c, op, compute), op).total));
   return need;
 }
 
@@ -628,12 +638,12 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
     const bool f32 = compute == HIMUON_FP32;
     Ops ops{compute, compute == HIMUON_FP16 ? HIMUON_FP16 : HIMUON_BF16, status_ptr(), stream};
     const int32_t dt16 = ops.op16;
-    const int64_t per = chunk_tiles(c, limit, compute, gram);
+    const int64_t per = chunk_tiles(c, limit, compute, op);
     if (per < 1) return HIMUON_ERR_WORKSPACE;
     const int64_t n = c.n, m = c.m;
     for (int64_t t0 = 0; t0 < static_cast<int64_t>(c.tiles.size()); t0 += per) {
       const int64_t bc = std::min<int64_t>(per, static_cast<int64_t>(c.tiles.size()) - t0);
-      const WsLayout L = ws_layout(n, m, bc, compute, gram);
+      const WsLayout L = ws_layout(n, m, bc, compute, op);
       float *x32[2] = {reinterpret_cast<float *>(W + L.x32a), f32 ? reinterpret_cast<float *>(W + L.x32b) : nullptr};
       void *x16[2] = {f32 ? nullptr : W + L.x16a, f32 ? nullptr : W + L.x16b};
       float *a32 = (f32 || gram) ? reinterpret_cast<float *>(W + L.a32) : nullptr;
@@ -643,10 +653,11 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       // step's two products over X apply 1 / rho^2 and 1 / rho in their
       // epilogues (no normalisation pass, no fp32 copy of the input).  fp16
       // keeps the pass: an unnormalised input may not fit fp16's range.
-      const bool prescale = !f32 && !gram && dt16 == HIMUON_BF16;
+      const bool prescale = staged_prescale(compute, op);
+      const bool two_pass = staged_two_pass(compute, op);
       float *inv = reinterpret_cast<float *>(W + L.scale), *inv2 = inv + bc;
-      if (c.padded) {
-        if (prescale) HIMUON_TRY(cudaMemsetAsync(x16[0], 0, 2 * n * m * bc, stream));
+      if (c.padded) {   // the zero padding of ragged tiles (pack writes the valid part only)
+        if (prescale || two_pass) HIMUON_TRY(cudaMemsetAsync(x16[0], 0, 2 * n * m * bc, stream));
         else HIMUON_TRY(cudaMemsetAsync(x32[0], 0, sizeof(float) * n * m * bc, stream));
       }
       PackArgs pk;
@@ -655,26 +666,36 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       pk.n_tiles = bc;
       pk.n = n;
       pk.m = m;
-      pk.x32 = prescale ? nullptr : x32[0];
-      pk.x16 = prescale ? x16[0] : nullptr;
+      pk.x32 = (prescale || two_pass) ? nullptr : x32[0];
+      pk.x16 = prescale ? x16[0] : nullptr;   // two_pass: sums of squares only, first
+      pk.x16_dtype = dt16;
+      pk.scale = nullptr;
       pk.partial = reinterpret_cast<float *>(W + L.partial);
       pk.parts = static_cast<int32_t>((std::max(n, m) + 31) / 32);
       pk.mode = step ? 1 : 0;
       pk.mu = mu;
       HIMUON_TRY(launch_pack(pk, stream));
-      NormArgs na;
-      na.n_tiles = bc;
-      na.elems = n * m;
-      na.x32 = x32[0];
-      na.x16 = x16[0];
-      na.x16_dtype = dt16;
-      na.partial = pk.partial;
-      na.parts = pk.parts;
-      na.keep32 = f32 ? 1 : 0;   // the 16-bit paths (NS and Gram NS) read only the 16-bit copy
-      na.eps = p.eps;
-      na.safety = safety;
-      if (prescale) HIMUON_TRY(launch_tile_scales(pk.partial, pk.parts, bc, p.eps, safety, inv, inv2, stream));
-      else HIMUON_TRY(launch_normalize(na, stream));
+      if (prescale || two_pass) {
+        HIMUON_TRY(launch_tile_scales(pk.partial, pk.parts, bc, p.eps, safety, inv, inv2, stream));
+        if (two_pass) {   // the scaled 16-bit operand from a second pass over the input
+          pk.x16 = x16[0];
+          pk.scale = inv;
+          HIMUON_TRY(launch_pack(pk, stream));
+        }
+      } else {
+        NormArgs na;
+        na.n_tiles = bc;
+        na.elems = n * m;
+        na.x32 = x32[0];
+        na.x16 = f32 ? nullptr : x16[0];
+        na.x16_dtype = dt16;
+        na.partial = pk.partial;
+        na.parts = pk.parts;
+        na.keep32 = f32 ? 1 : 0;   // the fp16 momentum step reads only the 16-bit copy
+        na.eps = p.eps;
+        na.safety = safety;
+        HIMUON_TRY(launch_normalize(na, stream));
+      }
       int cur = 0;  // which x buffer holds the current operand
       float *xfinal = x32[0];
       int rc = HIMUON_OK;
@@ -1014,13 +1035,12 @@ int64_t workspace_one(const CallMats &cm, const himuon_split *splits, const himu
   int64_t need = 0;
   std::vector<TileClass> classes;
   staged_classes(blocks, classes);
-  const bool gram = op == HIMUON_OP_GRAM_NS;
   for (const TileClass &c : classes) {
     const int compute = class_compute(c, op, p.compute);
     int64_t k = std::min<int64_t>(static_cast<int64_t>(c.tiles.size()), 65535);
-    int64_t bytes = static_cast<int64_t>(ws_layout(c.n, c.m, k, compute, gram).total);
+    int64_t bytes = static_cast<int64_t>(ws_layout(c.n, c.m, k, compute, op).total);
     if (p.chunk_bytes > 0 && bytes > p.chunk_bytes)
-      bytes = std::max<int64_t>(p.chunk_bytes, static_cast<int64_t>(ws_layout(c.n, c.m, 1, compute, gram).total));
+      bytes = std::max<int64_t>(p.chunk_bytes, static_cast<int64_t>(ws_layout(c.n, c.m, 1, compute, op).total));
     need = std::max(need, bytes);
   }
   return need;

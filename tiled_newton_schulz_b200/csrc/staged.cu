@@ -100,7 +100,8 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
   const int32_t i0 = blockIdx.x * rpp;
   const int32_t i1 = min(tl.h, i0 + rpp);
   float *x = a.x32 ? a.x32 + t * a.n * a.m : nullptr;
-  __nv_bfloat16 *xh = a.x32 ? nullptr : static_cast<__nv_bfloat16 *>(a.x16) + t * a.n * a.m;
+  void *xh = (a.x32 || !a.x16) ? nullptr : static_cast<void *>(static_cast<uint16_t *>(a.x16) + t * a.n * a.m);
+  const float sc = a.scale ? a.scale[t] : 1.f;
   float ss = 0.f;
   if (i0 < i1) {
     const void *src = b.ptr[kRoleIn];
@@ -128,16 +129,19 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
       if (xh) {
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = v[e] * sc;
         if (tl.transposed) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xh[static_cast<int64_t>(j + e) * a.m + i] = __float2bfloat16_rn(v[e]);
+          for (int e = 0; e < 8; ++e) st_elem(xh, a.x16_dtype, static_cast<int64_t>(j + e) * a.m + i, w[e]);
         } else {
-          st8_16(xh, HIMUON_BF16, static_cast<int64_t>(i) * a.m + j, v);
+          st8_16(xh, a.x16_dtype, static_cast<int64_t>(i) * a.m + j, w);
         }
-      } else if (tl.transposed) {
+      } else if (x && tl.transposed) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[static_cast<int64_t>(j + e) * a.m + i] = v[e];
-      } else {
+      } else if (x) {
         float4 *xo = reinterpret_cast<float4 *>(x + static_cast<int64_t>(i) * a.m + j);
         xo[0] = make_float4(v[0], v[1], v[2], v[3]);
         xo[1] = make_float4(v[4], v[5], v[6], v[7]);
@@ -153,12 +157,12 @@ __global__ void __launch_bounds__(256) pack_kernel(const PackArgs a) {
       }
       ss = fmaf(v, v, ss);
       const int64_t o = tl.transposed ? static_cast<int64_t>(j) * a.m + i : static_cast<int64_t>(i) * a.m + j;
-      if (xh) xh[o] = __float2bfloat16_rn(v);
-      else x[o] = v;
+      if (xh) st_elem(xh, a.x16_dtype, o, v * sc);
+      else if (x) x[o] = v;
     }
   }
   const float s = block_sum<256>(ss, scratch);
-  if (threadIdx.x == 0) a.partial[t * a.parts + blockIdx.x] = s;
+  if (threadIdx.x == 0 && !a.scale) a.partial[t * a.parts + blockIdx.x] = s;   // (the second pass: already summed)
 }
 
 // grid (chunks, tiles): rho from the partial sums (fixed order), then scale,

@@ -69,7 +69,10 @@ struct PackArgs {
   int64_t n_tiles;
   int64_t n, m;           // padded iterate shape (n <= m), row-major n x m per tile
   float *x32;             // n_tiles * n * m (fp32 iterate), or nullptr when x16 takes the values
-  void *x16;              // bf16 copy instead of x32 (the bf16 path scales in its first products)
+  void *x16;              // 16-bit copy instead of x32 (x16_dtype; neither: sums of squares only)
+  int32_t x16_dtype;
+  const float *scale;     // with x16: per-tile factor applied before rounding (the second pass
+                          // of a two-pass normalisation; nullptr: the values as they are)
   float *partial;         // n_tiles * parts
   int32_t parts;          // partial sums per tile (row slices of the source tile)
   int32_t mode;           // 0: NS input; 1: momentum (M' = mu M + G written back to M)
