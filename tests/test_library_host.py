@@ -101,6 +101,32 @@ def test_workspace_size_on_the_host(lib):
     assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(pc), 0) <= 64 << 20
 
 
+@pytest.mark.parametrize("op,compute,expect_mib", [
+    # 16-bit operand ping-pong 2 x 8 MiB, A and Bop 2 x 2 MiB: no fp32 X (bf16 NS
+    # scales in its first products, fp16 NS writes the scaled operand in a second
+    # pass over the input, and both last products write the caller's buffer)
+    (himuon.OP_NS_FULL, himuon.BF16, 20),
+    (himuon.OP_NS_FULL, himuon.FP16, 20),
+    (himuon.OP_MOMENTUM_STEP, himuon.BF16, 20),
+    # the fp16 momentum step normalises from an fp32 X (16 MiB)
+    (himuon.OP_MOMENTUM_STEP, himuon.FP16, 36),
+    # Gram NS in fp16: operands 16, R fp32 + fp16 6, RZ fp32 4, Q x 2, Z, RZ fp16 8
+    (himuon.OP_GRAM_NS, himuon.FP16, 34),
+    # fp32: X x 2 32, A and B 8; Gram adds RZ, Q, Z, a second Q (fp32)
+    (himuon.OP_NS_FULL, himuon.FP32, 40),
+    (himuon.OP_GRAM_NS, himuon.FP32, 52),
+])
+def test_staged_workspace_layout_on_the_host(lib, op, compute, expect_mib):
+    """The staged workspace of one 1024 x 4096 matrix, whole (n = 1024, m =
+    4096, one tile), buffer by buffer: a path that reads the fp32 X must have
+    one of its own (its offset would otherwise alias the 16-bit operand), and
+    the paths that never touch it must not pay for it.  768 B of per-tile
+    partial sums and scales come on top."""
+    mats = (himuon.Mat * 1)(himuon.Mat(0x1000, 1024, 4096, 4096, himuon.BF16))
+    p = himuon.params(0, (3.4445, -4.7750, 2.0315), steps=5, compute=compute, restart=(3,) if op == himuon.OP_GRAM_NS else ())
+    assert lib.himuon_workspace_size(mats, 1, None, ctypes.byref(p), op) == expect_mib * (1 << 20) + 768
+
+
 def test_per_matrix_tiles_on_the_host(lib):
     """p->tiles: the workspace is the largest group's need; the fixed-scratch
     entry point rejects it; a bad matrix in any group fails the whole call."""
