@@ -752,9 +752,11 @@ int run_staged(const Plan &plan, int op, const himuon_ns_params &p, float mu, fl
       } else {
         // Gram NS (Algorithm 3): R = X X^T, Q = I; restarts X <- Q X.  The terms
         // a R, a RZ stay fp32 (C operands): folding a I into a 16-bit Z, or
-        // reading R or RZ rounded to 16 bits, loses R's small eigen-directions
-        // (below fp16's normal range), which later steps feed back (fp16 R and
-        // RZ terms: 4.6% error on a 256 x 1024 input without a restart).  The
+        // reading R or RZ rounded to 16 bits, loses R's small eigen-directions,
+        // which later steps feed back (fp16 R and RZ terms: 4.6% error on a
+        // 256 x 1024 input without a restart).  It is fp16's precision, not its
+        // range: the same copies scaled by 2^8 .. 2^14, all entries normal,
+        // lose as much.  The
         // a Q term reads the 16-bit Q: Q's eigenvalues stay of the order of a
         // or above and Q is never fed back into R, so its rounding costs
         // nothing (equal or smaller errors under every restart pattern tried,
