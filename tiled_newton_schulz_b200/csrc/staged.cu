@@ -385,25 +385,17 @@ __device__ __forceinline__ void epi_scatter8(const EpiArgs &e, const ScatterDst 
   }
 }
 
-// Write 8 consecutive outputs starting at element index `o` of the batch;
-// they sit in row `row`, columns col..col+7 of their matrix.  With `mirror`
-// (an off-diagonal tile of a symmetric product) they also go to rows
-// col..col+7, column `row` (element index `om` for the first; a warp's lanes
-// hold consecutive rows, so each of these scalar stores is coalesced).
-// `alpha` is the product's alpha for this matrix and `sd`, with the scatter
-// epilogue, its destination (both resolved once per output tile).
-__device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t row, int64_t col, const float *acc,
-                                           bool mirror, int64_t om, float alpha, const ScatterDst &sd) {
-  float v[8];
+// The C term's 8 values at element index `o` of the batch (c32, or c16 in
+// out16_dtype), loaded ahead of the accumulator so that a group's loads are in
+// flight together.
+__device__ __forceinline__ void epi_load_c8(const EpiArgs &e, int64_t o, float *cc) {
   if (e.c32) {
     const float4 c0 = *reinterpret_cast<const float4 *>(e.c32 + o);
     const float4 c1 = *reinterpret_cast<const float4 *>(e.c32 + o + 4);
-    const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = fmaf(alpha, acc[i], e.beta * cc[i]);
-  } else if (e.c16) {
+    cc[0] = c0.x; cc[1] = c0.y; cc[2] = c0.z; cc[3] = c0.w;
+    cc[4] = c1.x; cc[5] = c1.y; cc[6] = c1.z; cc[7] = c1.w;
+  } else {
     const uint4 u = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(e.c16) + o);
-    float cc[8];
     if (e.out16_dtype == HIMUON_FP16) {
       const __half2 *h = reinterpret_cast<const __half2 *>(&u);
 #pragma unroll
@@ -421,6 +413,22 @@ __device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t 
         cc[2 * i + 1] = f.y;
       }
     }
+  }
+}
+
+// Write 8 consecutive outputs starting at element index `o` of the batch;
+// they sit in row `row`, columns col..col+7 of their matrix.  With `mirror`
+// (an off-diagonal tile of a symmetric product) they also go to rows
+// col..col+7, column `row` (element index `om` for the first; a warp's lanes
+// hold consecutive rows, so each of these scalar stores is coalesced).
+// `alpha` is the product's alpha for this matrix, `cc` the C term's values
+// (epi_load_c8; nullptr: none) and `sd`, with the scatter epilogue, the
+// matrix's destination (alpha and sd resolved once per output tile).
+__device__ __forceinline__ void epi_store8(const EpiArgs &e, int64_t o, int64_t row, int64_t col, const float *acc,
+                                           bool mirror, int64_t om, float alpha, const float *cc,
+                                           const ScatterDst &sd) {
+  float v[8];
+  if (cc) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = fmaf(alpha, acc[i], e.beta * cc[i]);
   } else {
@@ -611,6 +619,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;                    // TMEM lanes 32 q .. 32 q + 31
     const int half = (warp - 2) >> 2;          // columns half * BN / 2 ..
     const int row = q * 32 + lane;
+    const bool has_c = a.ep.c32 || a.ep.c16;
     int64_t j = 0;
     for (int64_t idx = blockIdx.x; idx < a.n_tiles; idx += gridDim.x, ++j) {
       const int b = static_cast<int>(j & 1);
@@ -629,6 +638,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int32_t ct = (n0 + 32 * i) / 128;   // 128-column block of the output
         if (a.ep.sym && ct > ti) break;          // above the diagonal (the tile's last block)
         const bool mirror = a.ep.sym && ct < ti;
+        // the group's C loads first, all four in flight (issued one by one
+        // between the stores, each waited for its own trip to memory)
+        float cv[32];
+        if (has_c) {
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) epi_load_c8(a.ep, obase + 32 * i + 8 * jj, cv + 8 * jj);
+        }
         float v[32];
         tmem_ld32(taddr + 32 * i, v);
         tmem_wait_ld();
@@ -636,7 +652,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int jj = 0; jj < 4; ++jj) {
           const int64_t col = n0 + 32 * i + 8 * jj;
           epi_store8(a.ep, obase + 32 * i + 8 * jj, m0 + row, col, v + 8 * jj, mirror,
-                     z * a.ep.stride + col * a.ep.N + m0 + row, alpha, sd);
+                     z * a.ep.stride + col * a.ep.N + m0 + row, alpha, has_c ? cv + 8 * jj : nullptr, sd);
         }
       }
       tc_fence_before();
