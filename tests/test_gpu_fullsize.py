@@ -212,3 +212,23 @@ def test_moe_experts_gram_and_standard_sampled(hm):
             got = f64(Y[k])
             assert rel(got, ref) <= TOL16
             assert svd_dev(got, ref) <= SVTOL
+
+
+def test_gram_and_fp16_ns_2048x4096_against_oracle(hm):
+    """One 2048 x 4096 matrix: Gram NS (fp16, restart at t = 3) and standard NS
+    with fp16 operands.  At n >= 2048 the symmetric n x n products run on
+    128 x 256 tiles, with Gram's fp32 terms kept on and below the diagonal,
+    its Q in fp16, and fp16 NS's operand written by the second pass over the
+    input; the 64-expert test (n = 1024) reaches none of that with 256-column
+    tiles.  Both outputs are compared with the oracle's Gram NS, which equals
+    its standard NS to ~1e-14 (pinned on the CPU)."""
+    x = inputs.gaussian_torch(2048, 4096, 2048, "cuda")
+    yg, ys = torch.empty_like(x), torch.empty_like(x)
+    hm.gram_ns([x], [yg], hm.params(0, QUINTIC, steps=5, compute=hm.FP16, restart=(3,)))
+    hm.ns_full([x], [ys], hm.params(0, QUINTIC, steps=5, compute=hm.FP16))
+    assert hm.device_status() == 0
+    ref = oracle.gram_ns(f64(x), C32, restart=(3,))
+    for y in (yg, ys):
+        got = f64(y)
+        assert rel(got, ref) <= TOL16
+        assert svd_dev(got, ref) <= SVTOL
