@@ -217,8 +217,9 @@ HIMUON_API int himuon_version(void);
  * exits.  The call allocates no device memory (no cudaMalloc, cudaFree or
  * allocating library routine) and bypasses the plan cache.  A call whose
  * largest tile (or its tables) does not fit returns HIMUON_ERR_TOO_LARGE
- * before enqueuing anything; e.g. full-matrix NS fits up to about 1024 x 2048
- * in bf16 and 1024 x 1024 in fp32.
+ * before enqueuing anything; e.g. full-matrix NS of a 1024-row matrix fits up
+ * to 1024 x 7040 in bf16 (4 bytes of scratch per element plus 4 n^2 bytes for
+ * the n x n products) and 1024 x 2944 in fp32 (twice that).
  *
  * The first call on a device looks up that device's address of the array
  * (cudaGetSymbolAddress, with the device current) and keeps it for later
